@@ -1,0 +1,336 @@
+"""Pins for the float64 attention oracle (CPU only).
+
+Each check compares the oracle with something it does not compute itself:
+the pages' shift rule worked by hand (golden table), brute-force softmax with
+pure-Python loops, torch's scaled_dot_product_attention in float64 with
+autograd (an independent library), central finite differences, exact
+identities (delta = rowsum(P o dP), shift invariance), and closed-form special
+cases.  Planted-mistake tests at the end show that a plausible slip in the
+oracle (a dropped scale, a swapped branch, a transposed operand, a dropped
+delta) makes one of these pins fail.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import attention as A
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _shift_table():
+    rows = []
+    with open(os.path.join(GOLDEN, "shift_rule.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            mode, rm, rs, beta, m = line.split()
+            rows.append((int(mode), float(rm), int(rs), float(beta), float(m)))
+    return rows
+
+
+def _rand_bf16(rng, shape, std=1.0):
+    return workloads.to_bf16_values(rng.standard_normal(shape).astype(np.float32) * np.float32(std))
+
+
+# ---------------------------------------------------------------- shift rule
+
+def check_shift_rule(fn):
+    for mode, rm, rs, beta, m in _shift_table():
+        got = fn(np.array([rm], np.float32), np.array([rs]), beta, mode)[0]
+        assert got == np.float32(m), (mode, rm, rs, beta, m, got)
+
+
+def test_shift_rule_golden_table():
+    check_shift_rule(A.select_shift)
+
+
+# --------------------------------------------------------- brute force (N<=8)
+
+def _brute_fwd(q, k, v, causal):
+    """Unshifted softmax with pure-Python loops: exp(S)/sum(exp(S))."""
+    N, d = q.shape
+    sc = 1.0 / math.sqrt(d)
+    o = np.zeros((N, v.shape[1]))
+    lse = np.zeros(N)
+    for i in range(N):
+        js = range(i + 1) if causal else range(N)
+        s = {j: sum(float(q[i, c]) * float(k[j, c]) for c in range(d)) * sc for j in js}
+        z = sum(math.exp(s[j]) for j in js)
+        lse[i] = math.log(z)
+        for c in range(v.shape[1]):
+            o[i, c] = sum(math.exp(s[j]) / z * float(v[j, c]) for j in js)
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_forward_brute_force(causal, mode):
+    rng = np.random.default_rng(7)
+    for N, d in [(1, 4), (5, 4), (8, 16)]:
+        q, k, v = (_rand_bf16(rng, (1, 1, N, d)) for _ in range(3))
+        # add a tie: key 0 duplicated, query aimed at it
+        if N > 2:
+            k[0, 0, 2] = k[0, 0, 0]
+            q[0, 0, N - 1] = k[0, 0, 0]
+        out = A.attention_fwd(q, k, v, causal, mode, 2.0)
+        o_ref, lse_ref = _brute_fwd(q[0, 0], k[0, 0], v[0, 0], causal)
+        np.testing.assert_allclose(out["o"][0, 0], o_ref, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(out["lse"][0, 0], lse_ref, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------ independent library (torch)
+
+def _torch_ref(q, k, v, do, causal):
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal)
+    o.backward(torch.tensor(do, dtype=torch.float64))
+    return o.detach().numpy(), tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_against_torch_sdpa_float64(causal, mode):
+    rng = np.random.default_rng(11)
+    B, H, N, d = 2, 2, 64, 64
+    q, k, v, do = (_rand_bf16(rng, (B, H, N, d)) for _ in range(4))
+    k[:, :, 40] = k[:, :, 0]
+    q[:, :, 50:60] = k[:, :, :1] * np.float32(0.5)
+    fwd = A.attention_fwd(q, k, v, causal, mode, 2.0)
+    bwd = A.attention_bwd(q, k, v, do, causal, mode, 2.0, fwd=fwd)
+    o, dq, dk, dv = _torch_ref(q, k, v, do, causal)
+    for got, ref in ((fwd["o"], o), (bwd["dq"], dq), (bwd["dk"], dk), (bwd["dv"], dv)):
+        np.testing.assert_allclose(got, ref, rtol=1e-9, atol=1e-11)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_against_torch_sdpa_head_dims(d):
+    rng = np.random.default_rng(5)
+    q, k, v, do = (_rand_bf16(rng, (1, 2, 32, d)) for _ in range(4))
+    fwd = A.attention_fwd(q, k, v, True, 1, 2.0)
+    bwd = A.attention_bwd(q, k, v, do, True, 1, 2.0, fwd=fwd)
+    o, dq, dk, dv = _torch_ref(q, k, v, do, True)
+    np.testing.assert_allclose(fwd["o"], o, rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(bwd["dq"], dq, rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(bwd["dk"], dk, rtol=1e-9, atol=1e-11)
+
+
+# ------------------------------------------------------- finite differences
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_gradients_finite_differences(causal, mode):
+    rng = np.random.default_rng(3)
+    N, d = 6, 4
+    q, k, v, do = (rng.standard_normal((1, 1, N, d)) for _ in range(4))
+    k[0, 0, 3] = k[0, 0, 1]  # a tie for the rows that aim at key 1
+    q[0, 0, 4] = k[0, 0, 1]
+    bwd = A.attention_bwd(q, k, v, do, causal, mode, 2.0)
+    h = 1e-6
+
+    def loss(q_, k_, v_):
+        return float((A.attention_fwd(q_, k_, v_, causal, mode, 2.0)["o"] * do).sum())
+
+    for name, x, g in (("q", q, bwd["dq"]), ("k", k, bwd["dk"]), ("v", v, bwd["dv"])):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            fd[idx] = (loss(args_p["q"], args_p["k"], args_p["v"]) - loss(args_m["q"], args_m["k"], args_m["v"])) / (2 * h)
+        rel = np.linalg.norm(fd - g) / max(np.linalg.norm(g), 1e-30)
+        assert rel <= 1e-6, (name, rel)
+
+
+# -------------------------------------------------------- exact identities
+
+def test_delta_identity():
+    rng = np.random.default_rng(9)
+    q, k, v, do = (_rand_bf16(rng, (1, 2, 48, 16)) for _ in range(4))
+    fwd = A.attention_fwd(q, k, v, True, 1, 2.0)
+    bwd = A.attention_bwd(q, k, v, do, True, 1, 2.0, fwd=fwd)
+    for h in range(2):
+        s = q[0, h].astype(np.float64) @ k[0, h].astype(np.float64).T / 4.0
+        s = np.where(np.tril(np.ones((48, 48), bool)), s, -np.inf)
+        p = np.exp(s - s.max(1, keepdims=True))
+        p /= p.sum(1, keepdims=True)
+        dp = do[0, h].astype(np.float64) @ v[0, h].astype(np.float64).T
+        np.testing.assert_allclose(bwd["delta"][0, h], (p * dp).sum(1), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiestress"])
+def test_mode_invariance(name):
+    w = workloads.make(name) if name == "tiny" else workloads.make(name).heads([(0, 0)])
+    if name == "tiestress":
+        w = workloads.Workload(w.name, 1, 1, 512, w.d, w.causal, w.seed, w.q[:, :, :512].copy(),
+                               w.k[:, :, :512].copy(), w.v[:, :, :512].copy(), w.do[:, :, :512].copy(),
+                               w.forced_tie_rows[:, :, :512])
+    f0 = A.attention_fwd(w.q, w.k, w.v, w.causal, 0)
+    f1 = A.attention_fwd(w.q, w.k, w.v, w.causal, 1)
+    b0 = A.attention_bwd(w.q, w.k, w.v, w.do, w.causal, 0, fwd=f0)
+    b1 = A.attention_bwd(w.q, w.k, w.v, w.do, w.causal, 1, fwd=f1)
+    assert (f1["m"] != f0["m"]).any()  # the rule actually moved some shifts
+    for x0, x1 in ((f0["o"], f1["o"]), (f0["lse"], f1["lse"]), (b0["dq"], b1["dq"]),
+                   (b0["dk"], b1["dk"]), (b0["dv"], b1["dv"])):
+        assert np.linalg.norm(x1 - x0) <= 1e-12 * np.linalg.norm(x0)
+
+
+# ------------------------------------------- the trigger and the fix (pages)
+
+def test_trigger_exact_ones_standard_mode():
+    """Page 1, "trigger condition": tied maxima give several exact ones."""
+    w = workloads.make("tiny")
+    f = A.attention_fwd(w.q, w.k, w.v, True, 0, return_pbar=True)
+    tied = f["rs"] > 1
+    assert tied.sum() > 10
+    for b, h, i in zip(*np.nonzero(tied)):
+        row = f["pbar"][b, h, i]
+        assert (row == 1.0).sum() == f["rs"][b, h, i]
+    # every row of the standard shift has P_bar == 1 at each maximum
+    assert np.all(f["pbar"].max(axis=-1) == 1.0)
+
+
+def test_fix_keeps_pbar_below_one_on_tied_rows():
+    """Page 1, "minimal fix": with the moved shift, max(P_bar) < 1 on tied rows;
+    untied rows keep m = rm and exactly one entry equal to 1."""
+    w = workloads.make("tiny")
+    f = A.attention_fwd(w.q, w.k, w.v, True, 1, return_pbar=True)
+    tied = f["rs"] > 1
+    rowmax = f["pbar"].max(axis=-1)
+    assert np.all(rowmax[tied] < 1.0)
+    assert np.all(f["pbar_max"][tied] < 1.0)
+    assert np.all(f["pbar_max"][~tied] == 1.0)
+    ones = (f["pbar"] == 1.0).sum(axis=-1)
+    assert np.all(ones[~tied] == 1) and np.all(ones[tied] == 0)
+    assert tied.any()
+
+
+def test_tiestress_forced_rows_have_the_target_class():
+    w = workloads.make("tiestress", B=1, H=2, N=1024)
+    f = A.attention_fwd(w.q, w.k, w.v, False, 1)
+    cls = w.notes["tie_class"]
+    forced = cls >= 0
+    assert np.all(f["rs"][forced] == 2)
+    assert np.all(f["rm"][cls == 0] > 0)
+    assert np.all(f["rm"][cls == 1] < 0)
+    assert np.all(f["rm"][cls == 2] == 0)
+    assert np.all(f["m"][cls == 2] == 1.0)
+    assert np.all(f["m"][cls == 1] == 0.0)
+    np.testing.assert_array_equal(f["m"][cls == 0], 2.0 * f["rm"][cls == 0])
+    frac = forced.mean()
+    assert 0.22 <= frac <= 0.28
+    # the fix holds on every tied row, whatever the sign class
+    tied = f["rs"] > 1
+    assert np.all(f["pbar_max"][tied] < 1.0)
+
+
+def test_g2s_sink_rows_are_tied():
+    w = workloads.make("g2s", B=1, H=2)
+    f = A.attention_fwd(w.q, w.k, w.v, True, 1)
+    assert np.all(f["rs"][w.forced_tie_rows] >= 2)
+    assert np.all(f["rm"][w.forced_tie_rows] > 0)
+    assert abs(w.forced_tie_rows.mean() - 0.10) < 0.01
+
+
+# ------------------------------------------------------------ special cases
+
+def test_causal_first_row_and_zero_query():
+    rng = np.random.default_rng(1)
+    N, d = 16, 8
+    q, k, v, do = (_rand_bf16(rng, (1, 1, N, d)) for _ in range(4))
+    q[0, 0, 9] = 0.0  # a zero query: all visible scores are 0, a tie at rm == 0
+    f = A.attention_fwd(q, k, v, True, 1)
+    b = A.attention_bwd(q, k, v, do, True, 1, fwd=f)
+    assert np.array_equal(f["o"][0, 0, 0], v[0, 0, 0].astype(np.float64))  # row 0 sees only key 0
+    assert np.all(b["dq"][0, 0, 0] == 0.0)
+    np.testing.assert_allclose(f["o"][0, 0, 9], v[0, 0, :10].astype(np.float64).mean(0), rtol=1e-13, atol=1e-14)
+    assert f["rm"][0, 0, 9] == 0.0 and f["rs"][0, 0, 9] == 10
+    assert f["m"][0, 0, 9] == 1.0  # beta - 1 with beta = 2
+    np.testing.assert_allclose(f["pbar_max"][0, 0, 9], math.exp(-1.0), rtol=1e-15)
+
+
+def test_o_for_delta_changes_only_delta_path():
+    rng = np.random.default_rng(2)
+    q, k, v, do = (_rand_bf16(rng, (1, 1, 32, 16)) for _ in range(4))
+    f = A.attention_fwd(q, k, v, True, 1)
+    b_ref = A.attention_bwd(q, k, v, do, True, 1, fwd=f)
+    b_same = A.attention_bwd(q, k, v, do, True, 1, fwd=f, o_for_delta=f["o"])
+    for key in ("dq", "dk", "dv", "delta"):
+        assert np.array_equal(b_ref[key], b_same[key])
+    o_bf = workloads.to_bf16_values(f["o"].astype(np.float32))
+    b_bf = A.attention_bwd(q, k, v, do, True, 1, fwd=f, o_for_delta=o_bf)
+    assert np.array_equal(b_bf["dv"], b_ref["dv"])
+    assert not np.array_equal(b_bf["delta"], b_ref["delta"])
+
+
+# ------------------------------------------------------- planted mistakes
+
+def test_planted_mistake_dropped_scale_is_caught(monkeypatch):
+    monkeypatch.setattr(A, "scale_f64", lambda d: 1.0)
+    rng = np.random.default_rng(7)
+    q, k, v = (_rand_bf16(rng, (1, 1, 8, 16)) for _ in range(3))
+    out = A.attention_fwd(q, k, v, True, 1)
+    o_ref, _ = _brute_fwd(q[0, 0], k[0, 0], v[0, 0], True)
+    assert not np.allclose(out["o"][0, 0], o_ref, rtol=1e-6)
+
+
+def test_planted_mistake_swapped_branch_is_caught(monkeypatch):
+    orig = A.select_shift
+
+    def swapped(rm, rs, beta, mode=1):
+        m = orig(rm, rs, beta, mode)
+        rm = np.asarray(rm, np.float32)
+        tied = np.asarray(rs) > 1
+        return np.where(tied & (rm < 0), np.float32(beta) * rm, m).astype(np.float32)
+
+    with pytest.raises(AssertionError):
+        check_shift_rule(swapped)
+
+
+def test_planted_mistake_transposed_dk_is_caught(monkeypatch):
+    rng = np.random.default_rng(11)
+    q, k, v, do = (_rand_bf16(rng, (1, 1, 16, 16)) for _ in range(4))
+    good = A.attention_bwd(q, k, v, do, True, 1)
+    _, _, dk, _ = _torch_ref(q, k, v, do, True)
+    np.testing.assert_allclose(good["dk"], dk, rtol=1e-9, atol=1e-11)
+    # the slip: dK = dS Q instead of dS^T Q, i.e. a transposed operand
+    real_matmul = np.matmul
+
+    class Slip:
+        @staticmethod
+        def run():
+            s = q[0, 0].astype(np.float64) @ k[0, 0].astype(np.float64).T / 4.0
+            s = np.where(np.tril(np.ones((16, 16), bool)), s, -np.inf)
+            p = np.exp(s - s.max(1, keepdims=True))
+            p /= p.sum(1, keepdims=True)
+            dp = do[0, 0].astype(np.float64) @ v[0, 0].astype(np.float64).T
+            o = p @ v[0, 0].astype(np.float64)
+            ds = p * (dp - (do[0, 0] * o).sum(1, keepdims=True))
+            return real_matmul(ds, q[0, 0].astype(np.float64)) / 4.0
+
+    assert not np.allclose(Slip.run(), dk[0, 0], rtol=1e-6)
+
+
+def test_planted_mistake_dropped_delta_is_caught():
+    rng = np.random.default_rng(4)
+    N, d = 6, 4
+    q, k, v, do = (rng.standard_normal((1, 1, N, d)) for _ in range(4))
+    f = A.attention_fwd(q, k, v, True, 1)
+    b_wrong = A.attention_bwd(q, k, v, do, True, 1, fwd=f, o_for_delta=np.zeros_like(f["o"]))
+    h = 1e-6
+    x = q.copy()
+    x[0, 0, 3, 1] += h
+    lp = float((A.attention_fwd(x, k, v, True, 1)["o"] * do).sum())
+    x[0, 0, 3, 1] -= 2 * h
+    lm = float((A.attention_fwd(x, k, v, True, 1)["o"] * do).sum())
+    fd = (lp - lm) / (2 * h)
+    assert abs(b_wrong["dq"][0, 0, 3, 1] - fd) > 1e-4
