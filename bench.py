@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Benchmark: causal attention fwd+bwd TFLOP/s on B200, stabilised softmax.
+
+One step = fa_fwd + fa_bwd (delta, main, dQ convert) on the GPT-2-small
+attention workload (B8 H12 N1024 d64, causal, beta = 2), inputs resident in
+HBM.  The inputs (50 MB) fit in the 126 MB L2, so L2 is flushed (a 256 MiB
+write) before every timed step; the flush is outside the CUDA-event intervals.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own copy of the
+workload (independent (batch, head) problems, no collective on the data path:
+weak scaling); the timed interval is the max over ranks.  `--impl reference`
+times the CPU float64 oracle on a bounded sample of the same workload.
+
+FLOP convention: forward 4*B*H*N^2*d, backward 2.5x forward, halved when
+causal; total 7*B*H*N^2*d for causal.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd+bwd TFLOP/s (causal) and % of B200 dense BF16 peak, stabilised mode"
+WORKLOAD = "g2s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ("bf16_numerics_b200/csrc/fa_ptx.cuh", "bf16_numerics_b200/csrc/fa_fwd.cuh",
+                  "bf16_numerics_b200/csrc/fa_bwd.cuh", "bf16_numerics_b200/csrc/fa_lib.cu")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--mode", type=int, default=1, help="0 standard shift, 1 stabilised shift")
+    ap.add_argument("--beta", type=float, default=2.0)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bounded oracle sample (seconds of CPU work)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (matching source hash); else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == src:
+                return float(parts[3])
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
+
+
+# --------------------------------------------------------------- oracle arm
+def cpu_oracle_sample(w, mode, beta, seconds):
+    """Time the float64 oracle fwd+bwd on (batch, head) pairs until about
+    `seconds` of CPU work; returns (flops_done, elapsed, heads, threads)."""
+    from oracle import attention as A
+    from threadpoolctl import threadpool_info
+
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
+    per_head = w.flops_total() / len(pairs)
+    done, t0 = 0, time.perf_counter()
+    while done < len(pairs):
+        sub = w.heads([pairs[done]])
+        f = A.attention_fwd(sub.q, sub.k, sub.v, sub.causal, mode, beta)
+        A.attention_bwd(sub.q, sub.k, sub.v, sub.do, sub.causal, mode, beta, fwd=f)
+        done += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    elapsed = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return per_head * done, elapsed, done, threads
+
+
+def workload_config(w, mode, beta):
+    return {"workload": f"{w.name}: GPT-2 small attention B{w.B} H{w.H} N{w.N} d{w.d} causal, "
+                        f"{'stabilised' if mode == 1 else 'standard'} shift (beta={beta})",
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "softmax_mode": "stabilized" if mode == 1 else "standard", "beta": beta,
+            "l2": "flushed before every timed step (256 MiB write, outside the timed intervals)",
+            "inputs": "seeded synthetic N(0,1) Q,K,V,dO; key 0 duplicated, 10% of rows tied on it; V cols 0-7 mean -0.75"}
+
+
+def run_reference(args, rank, world):
+    import workloads
+
+    if rank != 0:
+        return 0
+    w = workloads.make(WORKLOAD)
+    per_step = min(1.0, 120.0 / max(1, args.steps + args.warmup))  # whole run bounded to ~2 min (>= 1 head/step)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, args.mode, args.beta, per_step)
+    flops, secs, heads = 0.0, 0.0, 0
+    threads = 1
+    for _ in range(args.steps):
+        f_, s_, h_, threads = cpu_oracle_sample(w, args.mode, args.beta, per_step)
+        flops += f_
+        secs += s_
+        heads += h_
+    value = flops / secs / 1e12
+    sample = (f"{heads} (b,h) heads of {w.B * w.H} over {args.steps} steps, float64 NumPy oracle fwd+bwd, "
+              f"throughput scaled per head")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, args.mode, args.beta),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import bf16_numerics_b200 as fa
+    import workloads
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = workloads.make(WORKLOAD, seed=workloads.CONFIGS[WORKLOAD][5] + rank)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    mode, beta, causal = args.mode, args.beta, w.causal
+
+    h_in = [torch.from_numpy(x).to(torch.bfloat16).pin_memory() for x in (w.q, w.k, w.v, w.do)]
+    q, k, v, do = (t.to(dev) for t in h_in)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, N, device=dev, dtype=torch.float32)
+    stats = fa.RowStats(m=torch.empty(B, H, N, device=dev, dtype=torch.float32))
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), device=dev, dtype=torch.uint8)
+    flush = torch.empty(256 * 1024 * 1024, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fa_fwd(q, k, v, o, lse, stats, causal, mode, beta, stream)
+        fa.fa_bwd(q, k, v, o, do, lse, stats.m, dq, dk, dv, ws, causal, mode, beta, stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    status, word = fa.fa_device_error()
+    if status != 0:
+        raise RuntimeError(f"device error word {word:#x} during warm-up")
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x for x in visible.split(",") if x.strip()]
+    phys = int(ids[local_rank]) if len(ids) > local_rank and ids[local_rank].strip().isdigit() else local_rank
+    sampler = ClockSampler(phys)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.2)
+    fa.fa_timing_enable(True)
+    for i in range(K):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        stops[i].record(stream)
+    torch.cuda.synchronize(dev)
+    fa.fa_timing_enable(False)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    per_kernel = fa.fa_timing_read()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, stops)]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms_max = float(t.item())
+    status, word = fa.fa_device_error()
+    if status != 0:
+        raise RuntimeError(f"device error word {word:#x} during timing")
+
+    flops_step = w.flops_total()
+    value = world * flops_step * K / (total_ms_max * 1e-3) / 1e12
+
+    # -------- end to end through the public API with host buffers
+    E = args.e2e_steps
+    h_out = [torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+    h2d = sum(x.numel() * x.element_size() for x in h_in)
+    d2h = sum(x.numel() * x.element_size() for x in h_out)
+
+    def e2e_step():
+        for hs, dt in zip(h_in, (q, k, v, do)):
+            dt.copy_(hs, non_blocking=True)
+        step()
+        for hs, dt in zip(h_out, (o, dq, dk, dv)):
+            hs.copy_(dt, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * flops_step * E / (float(te.item()) * 1e-3) / 1e12
+
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    peak_tf = float(peaks["bf16_tflops"])
+    hbm = float(peaks["hbm_gbs"])
+    # per-kernel roofline from the library's event records (launching stream)
+    fwd_flops = w.flops_fwd()
+    bwd_flops = 2.5 * fwd_flops
+    rows = B * H * N
+    delta_bytes = rows * d * 2 * 2 + rows * 4 + rows * d * 4  # read O, dO; write delta; clear dQ accumulator
+    dq_bytes = rows * d * 4 + rows * d * 2
+    kern = {}
+    for name, (n_l, ms) in per_kernel.items():
+        if n_l == 0:
+            continue
+        avg_s = ms / n_l * 1e-3
+        if name == "fa_fwd_kernel":
+            kern[name] = {"bound": "tensor", "avg_us": avg_s * 1e6, "achieved": fwd_flops / avg_s / 1e12,
+                          "unit": "TFLOP/s", "frac": fwd_flops / avg_s / 1e12 / peak_tf}
+        elif name == "fa_bwd_main_kernel":
+            kern[name] = {"bound": "tensor", "avg_us": avg_s * 1e6, "achieved": bwd_flops / avg_s / 1e12,
+                          "unit": "TFLOP/s", "frac": bwd_flops / avg_s / 1e12 / peak_tf}
+        elif name == "fa_bwd_delta_kernel":
+            kern[name] = {"bound": "hbm", "avg_us": avg_s * 1e6, "achieved": delta_bytes / avg_s / 1e9,
+                          "unit": "GB/s", "frac": delta_bytes / avg_s / 1e9 / hbm}
+        else:
+            kern[name] = {"bound": "hbm", "avg_us": avg_s * 1e6, "achieved": dq_bytes / avg_s / 1e9,
+                          "unit": "GB/s", "frac": dq_bytes / avg_s / 1e9 / hbm}
+        kern[name]["launches"] = n_l
+    dominant = max(per_kernel, key=lambda nm: per_kernel[nm][1])
+    dk_ = kern[dominant]
+    traffic = recorded_traffic(dominant)
+    roofline = {"kernel": dominant, "bound": dk_["bound"], "achieved": dk_["achieved"],
+                "peak": peak_tf if dk_["bound"] == "tensor" else hbm, "unit": dk_["unit"], "frac": dk_["frac"],
+                "traffic": traffic, "peak_source": f"{peak_src} ({'bf16_tflops burst' if dk_['bound'] == 'tensor' else 'hbm_gbs'})"}
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms_max / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w, mode, beta),
+            "pct_of_peak": 100.0 * value / (world * peak_tf),
+            "pct_of_sustained_peak": 100.0 * value / (world * float(peaks.get("bf16_tflops_sustained", peak_tf))),
+            "peak_source": peak_src,
+            "roofline": roofline, "kernels": kern, "gpu_launches": sum(n for n, _ in per_kernel.values()),
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": E, "outputs": "O, dQ, dK, dV copied back to pinned host memory"},
+            "clocks": clocks, "step_ms_p10_p50_p90": [float(np.percentile(step_ms, p)) for p in (10, 50, 90)]}
+    if world == 1 and not args.no_cpu_baseline:
+        flops_c, secs_c, heads_c, threads_c = cpu_oracle_sample(w, mode, beta, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": flops_c / secs_c / 1e12, "unit": "TFLOP/s", "cores": threads_c,
+                                "kind": "oracle",
+                                "sample": f"{heads_c} of {B * H} (b,h) heads of the same workload, float64 NumPy "
+                                          f"oracle fwd+bwd, {secs_c:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world != 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,330 @@
+// Host side of libfa_b200.so: argument validation, TMA tensor maps, kernel
+// launches, the device error word and optional per-kernel event timing.
+// The C ABI is declared (and documented) in include/fa_b200.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#include "fa_b200.h"
+#include "fa_bwd.cuh"
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+// [BH, N, D] bf16 -> 3-D tensor map, box 64 (d) x 128 (rows) x 1, 128B swizzle.
+// Rows past N read as zeros.
+bool make_map(CUtensorMap* map, const void* ptr, long long BH, long long N, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// ------------------------------------------------------------ event timing
+struct TimingRec {
+  int kernel;
+  cudaEvent_t start, stop;
+};
+bool g_timing = false;
+std::vector<TimingRec> g_recs;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+struct LaunchTimer {
+  int kernel;
+  cudaStream_t stream;
+  cudaEvent_t start = nullptr;
+  LaunchTimer(int k, cudaStream_t s) : kernel(k), stream(s) {
+    if (g_timing) {
+      start = take_event();
+      if (start) cudaEventRecord(start, stream);
+    }
+  }
+  void done() {
+    if (g_timing && start) {
+      cudaEvent_t stop = take_event();
+      if (stop) {
+        cudaEventRecord(stop, stream);
+        g_recs.push_back({kernel, start, stop});
+      } else {
+        g_event_pool.push_back(start);
+      }
+    }
+  }
+};
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+bool shape_ok(int B, int H, int N, int d) {
+  if (B < 0 || H < 0 || N < 0) return false;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH * N * d >= (1ll << 40)) return false;
+  const long long nblk = (static_cast<long long>(N) + 127) / 128;
+  if (BH * nblk >= (1ll << 31)) return false;
+  return true;
+}
+
+template <int D>
+fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const fa_row_stats* st,
+                     int BH, int N, int causal, int mode, float beta, cudaStream_t stream) {
+  using L = fa::FwdLayout<D>;
+  static bool attr = false;
+  if (!attr) {
+    if (!set_smem(fa::fa_fwd_kernel<D>, L::SMEM_BYTES)) return FA_ERR_CUDA;
+    attr = true;
+  }
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D)) return FA_ERR_CUDA;
+  fa::FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  if (st) {
+    p.st_rm = st->rm;
+    p.st_rs = st->rs;
+    p.st_m = st->m;
+    p.st_pbar_max = st->pbar_max;
+  }
+  p.BH = BH;
+  p.N = N;
+  p.n_qblk = (N + 127) / 128;
+  p.causal = causal;
+  p.mode = mode;
+  p.beta = beta;
+  p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_qblk) * BH);
+  LaunchTimer tm(FA_KERNEL_FWD, stream);
+  fa::fa_fwd_kernel<D><<<grid, 192, L::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  tm.done();
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int grid_for(long long work, int per_block) {
+  long long g = (work + per_block - 1) / per_block;
+  if (g > 148 * 16) g = 148 * 16;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+template <int D>
+fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                     const float* row_m, void* dq, void* dk, void* dv, uint8_t* ws, int BH, int N, int causal,
+                     int mode, cudaStream_t stream) {
+  using L = fa::BwdLayout<D>;
+  static bool attr = false;
+  if (!attr) {
+    if (!set_smem(fa::fa_bwd_main_kernel<D>, L::SMEM_BYTES)) return FA_ERR_CUDA;
+    attr = true;
+  }
+  const long long rows = static_cast<long long>(BH) * N;
+  float* delta = reinterpret_cast<float*>(ws);
+  float* dq_acc = reinterpret_cast<float*>(ws + round256(static_cast<size_t>(rows) * 4));
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D) ||
+      !make_map(&mdo, dO, BH, N, D))
+    return FA_ERR_CUDA;
+  {
+    constexpr int rows_per_block = 8 * (32 / (D / 8));
+    LaunchTimer tm(FA_KERNEL_BWD_DELTA, stream);
+    fa::fa_bwd_delta_kernel<D><<<grid_for(rows, rows_per_block), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows);
+    tm.done();
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  {
+    fa::BwdParams p{};
+    p.lse = lse;
+    p.row_m = row_m;
+    p.delta = delta;
+    p.dq_acc = dq_acc;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.BH = BH;
+    p.N = N;
+    p.n_blk = (N + 127) / 128;
+    p.causal = causal;
+    p.mode = mode;
+    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_blk) * BH);
+    LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
+    fa::fa_bwd_main_kernel<D><<<grid, 320, L::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
+    tm.done();
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  {
+    const long long n8 = rows * D / 8;
+    LaunchTimer tm(FA_KERNEL_BWD_DQ, stream);
+    fa::fa_bwd_dq_convert_kernel<<<grid_for(n8, 256), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
+                                                                         n8);
+    tm.done();
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported shape or head dimension";
+    case FA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case FA_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case FA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+  }
+  return "unknown status";
+}
+
+size_t fa_bwd_workspace_delta_offset(int B, int H, int N, int d) {
+  (void)B; (void)H; (void)N; (void)d;
+  return 0;
+}
+
+size_t fa_bwd_workspace_dq_offset(int B, int H, int N, int d) {
+  if (!shape_ok(B, H, N, d)) return 0;
+  return round256(static_cast<size_t>(B) * H * N * 4);
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (!shape_ok(B, H, N, d) || (d != 64 && d != 128)) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return round256(rows * 4) + round256(rows * static_cast<size_t>(d) * 4);
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const fa_row_stats* stats, int B,
+                 int H, int N, int d, int causal, int softmax_mode, float beta, void* stream) {
+  if (!shape_ok(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if (softmax_mode != FA_SOFTMAX_STANDARD && softmax_mode != FA_SOFTMAX_STABILIZED) return FA_ERR_INVALID_ARG;
+  if (softmax_mode == FA_SOFTMAX_STABILIZED && !(std::isfinite(beta) && beta > 1.0f)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N == 0) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (stats) {
+    const void* ptrs[4] = {stats->rm, stats->rs, stats->m, stats->pbar_max};
+    for (const void* sp : ptrs)
+      if (sp && (reinterpret_cast<uintptr_t>(sp) & 3u)) return FA_ERR_INVALID_ARG;
+  }
+  const int BH = B * H;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_fwd<64>(q, k, v, o, lse, stats, BH, N, causal, softmax_mode, beta, s);
+  return launch_fwd<128>(q, k, v, o, lse, stats, BH, N, causal, softmax_mode, beta, s);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 const float* row_m, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
+                 int H, int N, int d, int causal, int softmax_mode, float beta, void* stream) {
+  if (!shape_ok(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if (softmax_mode != FA_SOFTMAX_STANDARD && softmax_mode != FA_SOFTMAX_STABILIZED) return FA_ERR_INVALID_ARG;
+  if (softmax_mode == FA_SOFTMAX_STABILIZED && !(std::isfinite(beta) && beta > 1.0f)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N == 0) return FA_OK;
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (softmax_mode == FA_SOFTMAX_STABILIZED && !row_m) return FA_ERR_INVALID_ARG;
+  const void* a16[8] = {q, k, v, o, dO, dq, dk, dv};
+  for (const void* pp : a16)
+    if (!aligned16(pp)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (row_m && (reinterpret_cast<uintptr_t>(row_m) & 3u)))
+    return FA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d))
+    return FA_ERR_WORKSPACE;
+  const int BH = B * H;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, dO, lse, row_m, dq, dk, dv, ws, BH, N, causal, softmax_mode, s);
+  return launch_bwd<128>(q, k, v, o, dO, lse, row_m, dq, dk, dv, ws, BH, N, causal, softmax_mode, s);
+}
+
+fa_status fa_device_error(unsigned int* code) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_fa_error, sizeof(v)) != cudaSuccess) return FA_ERR_CUDA;
+  if (code) *code = v;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(fa::g_fa_error, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+fa_status fa_timing_enable(int enable) {
+  g_timing = enable != 0;
+  return FA_OK;
+}
+
+fa_status fa_timing_read(int* launches, double* total_ms) {
+  if (!launches || !total_ms) return FA_ERR_INVALID_ARG;
+  for (int i = 0; i < FA_NUM_KERNELS; ++i) {
+    launches[i] = 0;
+    total_ms[i] = 0.0;
+  }
+  fa_status st = FA_OK;
+  for (const TimingRec& r : g_recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+      st = FA_ERR_CUDA;
+    } else if (r.kernel >= 0 && r.kernel < FA_NUM_KERNELS) {
+      launches[r.kernel] += 1;
+      total_ms[r.kernel] += ms;
+    }
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  g_recs.clear();
+  return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+"""Shared helpers for the GPU parity tests: run the CUDA path through the C ABI
+on a workload, run the oracle on the same inputs (all heads or a sample), and
+compare with the tolerances the tests state.
+
+Tolerances (floating point): for O, dQ, dK, dV
+    max |gpu - ref| <= 1e-2 * max |ref|   and   ||gpu - ref||_F <= 5e-3 * ||ref||_F
+lse: |gpu - ref| <= 1e-3.  Integer / selection outputs (rm, rs, m) are compared
+bit for bit where S is exact in fp32 (inputs on a dyadic grid with d = 64);
+elsewhere rs and the branch of the shift rule must match and rm agrees to
+fp32 accumulation-order rounding.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import bf16_numerics_b200 as fa
+from oracle import attention as A
+
+MAXABS = 1e-2
+FROB = 5e-3
+LSE_ABS = 1e-3
+
+
+def to_dev(x: np.ndarray, dev) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(dev)
+
+
+def run_gpu(w, mode: int, beta: float = 2.0, dev="cuda:0", bwd: bool = True):
+    q, k, v, do = (to_dev(x, dev) for x in (w.q, w.k, w.v, w.do))
+    o, lse, st = fa.attention_forward(q, k, v, w.causal, mode, beta)
+    out = {"o": o, "lse": lse, "rm": st.rm, "rs": st.rs, "m": st.m, "pbar_max": st.pbar_max}
+    if bwd:
+        dq, dk, dv, ws = fa.attention_backward(q, k, v, o, do, lse, st.m, w.causal, mode, beta)
+        off_delta, _ = fa.fa_bwd_workspace_offsets(*q.shape)
+        B, H, N, _ = q.shape
+        delta = ws[off_delta:off_delta + B * H * N * 4].view(torch.float32).view(B, H, N)
+        out.update(dq=dq, dk=dk, dv=dv, delta=delta)
+    torch.cuda.synchronize(dev)
+    status, word = fa.fa_device_error()
+    assert status == 0, f"device error word {word:#x}"
+    return {k_: v_.float().cpu().numpy() if v_.dtype != torch.int32 else v_.cpu().numpy() for k_, v_ in out.items()}
+
+
+def head_slice(x, pairs):
+    return np.stack([x[b, h] for b, h in pairs])[None]
+
+
+def oracle(w, mode, beta=2.0, pairs=None, o_gpu=None):
+    if pairs is not None:
+        w = w.heads(pairs)
+    f = A.attention_fwd(w.q, w.k, w.v, w.causal, mode, beta)
+    b = A.attention_bwd(w.q, w.k, w.v, w.do, w.causal, mode, beta, fwd=f)
+    res = dict(f)
+    res.update(b)
+    if o_gpu is not None:
+        bd = A.attention_bwd(w.q, w.k, w.v, w.do, w.causal, mode, beta, fwd=f, o_for_delta=o_gpu)
+        res["delta_from_gpu_o"] = bd["delta"]
+    return res
+
+
+def assert_close(name, got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    scale = np.abs(ref).max()
+    maxerr = np.abs(got - ref).max()
+    frob = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert maxerr <= MAXABS * max(scale, 1e-30), f"{name}: max abs err {maxerr:.3e} > {MAXABS} * {scale:.3e}"
+    assert frob <= FROB, f"{name}: relative Frobenius err {frob:.3e} > {FROB}"
+    return maxerr / max(scale, 1e-30), frob
+
+
+def compare(gpu, ref, exact_stats: bool, pairs=None):
+    """gpu: dict of full-size arrays; ref: oracle on `pairs` (or all heads)."""
+    sel = (lambda x: head_slice(x, pairs)) if pairs is not None else (lambda x: x)
+    errs = {}
+    for key in ("o", "dq", "dk", "dv"):
+        if key in gpu:
+            errs[key] = assert_close(key, sel(gpu[key]), ref[key])
+    lse_err = np.abs(sel(gpu["lse"]) - ref["lse"]).max()
+    assert lse_err <= LSE_ABS, f"lse: max abs err {lse_err:.3e}"
+    if "delta" in gpu and "delta_from_gpu_o" in ref:
+        d_ref = ref["delta_from_gpu_o"]
+        d_err = np.abs(sel(gpu["delta"]) - d_ref).max()
+        assert d_err <= 1e-4 * max(np.abs(d_ref).max(), 1.0), f"delta: max abs err {d_err:.3e}"
+    rs_g, rs_r = sel(gpu["rs"]), ref["rs"]
+    if exact_stats:
+        assert np.array_equal(sel(gpu["rm"]), ref["rm"]), "rm not bit-exact"
+        assert np.array_equal(rs_g, rs_r), "rs not bit-exact"
+        assert np.array_equal(sel(gpu["m"]), ref["m"]), "m not bit-exact"
+    else:
+        assert np.array_equal(rs_g, rs_r), "rs differs"
+        rm_g, rm_r = sel(gpu["rm"]), ref["rm"]
+        np.testing.assert_allclose(rm_g, rm_r, rtol=1e-5, atol=1e-5)
+        branch = lambda rm, rs: np.where(rs > 1, np.sign(rm), 2)
+        assert np.array_equal(branch(rm_g, rs_g), branch(rm_r, rs_r)), "shift-rule branch differs"
+        np.testing.assert_allclose(sel(gpu["m"]), ref["m"], rtol=1e-5, atol=1e-5)
+    return errs

@@ -110,6 +110,8 @@ def _sink_ties(rng, q, k, frac):
     """
     B, H, N, _ = q.shape
     tie = np.zeros((B, H, N), dtype=bool)
+    if N < 4:
+        return tie
     n_rows = max(1, int(round(frac * N)))
     for b in range(B):
         for h in range(H):
