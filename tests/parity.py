@@ -3,8 +3,16 @@ on a workload, run the oracle on the same inputs (all heads or a sample), and
 compare with the tolerances the tests state.
 
 Tolerances (floating point): for O, dQ, dK, dV
-    max |gpu - ref| <= 1e-2 * max |ref|   and   ||gpu - ref||_F <= 5e-3 * ||ref||_F
-lse: |gpu - ref| <= 1e-3.  Integer / selection outputs (rm, rs, m) are compared
+    max |gpu - ref| <= 1e-2 * max |ref| + 1e-5   and   ||gpu - ref||_F <= 5e-3 * ||ref||_F
+(the 1e-5 absolute term only matters where the exact result is zero, e.g. dQ
+of a row that sees a single key); lse: |gpu - ref| <= 1e-3.
+
+The backward is an operation on (Q, K, V, O, dO, lse): its delta is
+rowsum(dO o O) of the O it is given.  The backward reference is therefore the
+oracle's backward evaluated on the O the GPU forward produced (bf16); the
+oracle's own float64 O gives the chained reference, whose difference from the
+given-O reference is the delta bias the pages describe (a bf16-rounded O
+entering delta), reported separately.  Integer / selection outputs (rm, rs, m) are compared
 bit for bit where S is exact in fp32 (inputs on a dyadic grid with d = 64);
 elsewhere rs and the branch of the shift rule must match and rm agrees to
 fp32 accumulation-order rounding.
@@ -19,6 +27,7 @@ import bf16_numerics_b200 as fa
 from oracle import attention as A
 
 MAXABS = 1e-2
+ATOL = 1e-5
 FROB = 5e-3
 LSE_ABS = 1e-3
 
@@ -51,12 +60,16 @@ def oracle(w, mode, beta=2.0, pairs=None, o_gpu=None):
     if pairs is not None:
         w = w.heads(pairs)
     f = A.attention_fwd(w.q, w.k, w.v, w.causal, mode, beta)
-    b = A.attention_bwd(w.q, w.k, w.v, w.do, w.causal, mode, beta, fwd=f)
+    chained = A.attention_bwd(w.q, w.k, w.v, w.do, w.causal, mode, beta, fwd=f)
     res = dict(f)
-    res.update(b)
-    if o_gpu is not None:
-        bd = A.attention_bwd(w.q, w.k, w.v, w.do, w.causal, mode, beta, fwd=f, o_for_delta=o_gpu)
-        res["delta_from_gpu_o"] = bd["delta"]
+    if o_gpu is None:
+        res.update(chained)
+    else:
+        given = A.attention_bwd(w.q, w.k, w.v, w.do, w.causal, mode, beta, fwd=f, o_for_delta=o_gpu)
+        res.update(given)
+        res["delta_from_gpu_o"] = given["delta"]
+        for key in ("dq", "dk", "dv", "delta"):
+            res[key + "_chained"] = chained[key]
     return res
 
 
@@ -67,10 +80,36 @@ def assert_close(name, got, ref):
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
     scale = np.abs(ref).max()
     maxerr = np.abs(got - ref).max()
-    frob = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
-    assert maxerr <= MAXABS * max(scale, 1e-30), f"{name}: max abs err {maxerr:.3e} > {MAXABS} * {scale:.3e}"
-    assert frob <= FROB, f"{name}: relative Frobenius err {frob:.3e} > {FROB}"
+    assert maxerr <= MAXABS * scale + ATOL, f"{name}: max abs err {maxerr:.3e} > {MAXABS} * {scale:.3e} + {ATOL}"
+    nref = np.linalg.norm(ref)
+    frob = np.linalg.norm(got - ref) / nref if nref > 0 else 0.0
+    if nref > ATOL * np.sqrt(ref.size):
+        assert frob <= FROB, f"{name}: relative Frobenius err {frob:.3e} > {FROB}"
     return maxerr / max(scale, 1e-30), frob
+
+
+def bf16_ds_dq_floor(w, ref, o_gpu):
+    """max|dQ_emul - dQ_ref| / max|dQ_ref| where dQ_emul = bf16(dS) K * scale,
+    with P, dP and delta taken from float64/fp32 arithmetic (delta from the
+    given bf16 O) and only dS rounded to bf16: the part of the dQ error that
+    comes from the operand precision of the dQ product alone."""
+    from oracle import bf16
+
+    B, H, N, d = w.q.shape
+    sc = 1.0 / np.sqrt(d)
+    num = 0.0
+    for b in range(B):
+        for h in range(H):
+            q, k, v, do = (x[b, h].astype(np.float64) for x in (w.q, w.k, w.v, w.do))
+            s = q @ k.T * sc
+            if w.causal:
+                s = np.where(np.tril(np.ones((N, N), bool)), s, -np.inf)
+            p = np.exp(s - ref["lse"][b, h][:, None])
+            dlt = (do * np.asarray(o_gpu, np.float64)[b, h]).sum(1)
+            ds = p * (do @ v.T - dlt[:, None])
+            dq = bf16.round_bf16(ds.astype(np.float32)).astype(np.float64) @ k * sc
+            num = max(num, np.abs(dq - ref["dq"][b, h]).max())
+    return num / np.abs(ref["dq"]).max()
 
 
 def compare(gpu, ref, exact_stats: bool, pairs=None):
