@@ -31,7 +31,7 @@ KERNEL_NAMES = ("fa_fwd_kernel", "fa_bwd_delta_kernel", "fa_bwd_main_kernel", "f
 # every symbol include/fa_b200.h declares
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_workspace_delta_offset",
            "fa_bwd_workspace_dq_offset", "fa_status_string", "fa_device_error", "fa_timing_enable",
-           "fa_timing_read")
+           "fa_timing_read", "fa_bwd_noalloc")
 
 
 class FaRowStats(ctypes.Structure):

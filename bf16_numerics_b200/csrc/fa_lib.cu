@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "fa_b200.h"
@@ -328,3 +329,57 @@ fa_status fa_timing_read(int* launches, double* total_ms) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free backward (declared in fa_b200.h next to fa_bwd).
+//
+// For callers that cannot allocate device memory (a static memory plan fixed
+// at start-up, or a plug-in without an allocator of its own): the backward's
+// scratch -- delta followed by the fp32 dQ accumulator, laid out exactly as
+// fa_bwd's workspace -- lives in the file-scope array below.  Its name is a
+// host-side stand-in in host code, so the device address is looked up once
+// per device with cudaGetSymbolAddress (device current) and that address is
+// what the kernels receive.  Nothing here allocates.  The delta kernel clears
+// the dQ accumulator on every call; delta is overwritten in full.  All calls
+// share the array: overlapping calls race.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+fa_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                    const float* lse, const float* row_m, void* dq, void* dk, void* dv, int B, int H,
+                                    int N, int d, int causal, int softmax_mode, float beta, void* stream) {
+  if (!shape_ok(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (fa_bwd_workspace_bytes(B, H, N, d) > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const fa_status st = noalloc_scratch(&scratch);
+  if (st != FA_OK) return st;
+  return fa_bwd(q, k, v, o, dO, lse, row_m, dq, dk, dv, scratch, FA_NOALLOC_SCRATCH_BYTES, B, H, N, d, causal,
+                softmax_mode, beta, stream);
+}

@@ -125,6 +125,33 @@ enum { FA_KERNEL_FWD = 0, FA_KERNEL_BWD_DELTA = 1, FA_KERNEL_BWD_MAIN = 2, FA_KE
 fa_status fa_timing_enable(int enable);
 fa_status fa_timing_read(int* launches, double* total_ms);
 
+/* Allocation-free backward.  The paper has no counterpart: this entry point
+ * exists for callers that cannot allocate device memory themselves --
+ * runtimes that fix every device buffer at start-up under a static memory
+ * plan and forbid allocation afterwards, and plug-ins that are handed tensors
+ * by a host framework but own no allocator.  Such callers cannot provide the
+ * workspace fa_bwd asks for.
+ *
+ * Same arguments and results as fa_bwd without the workspace.  The scratch
+ * (delta and the fp32 dQ accumulator) lives in one static device array of
+ * FA_NOALLOC_SCRATCH_BYTES inside the library; every GPU that loads the
+ * library holds that array until the process exits.  A problem whose
+ * fa_bwd_workspace_bytes exceeds it is rejected with FA_ERR_WORKSPACE before
+ * anything is launched.  The call allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *
+ * The first call on a device looks up the array's device address on that
+ * device (cudaGetSymbolAddress, with the device current); make that first
+ * call before any stream capture.  All calls share the one array and it keeps
+ * the last call's contents (the dQ accumulator is cleared by the call itself
+ * before use), so calls that overlap on the GPU -- on different streams, or
+ * from different host threads -- race on it and must be serialised by the
+ * caller.  Returns FA_ERR_CUDA if the address lookup fails. */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, const float* row_m, void* dq, void* dk, void* dv, int B, int H, int N,
+                         int d, int causal, int softmax_mode, float beta, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
