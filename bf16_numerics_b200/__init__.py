@@ -32,7 +32,10 @@ __all__ = ["FaError", "STANDARD", "STABILIZED", "RowStats", "fa_fwd", "fa_bwd", 
 
 class FaError(RuntimeError):
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what}: {_abi.status_string(code)} (status {code})")
+        detail = ""
+        if code == _abi.FA_ERR_CUDA:
+            detail = " [" + _abi.load().fa_last_error_string().decode() + "]"
+        super().__init__(f"{what}: {_abi.status_string(code)} (status {code}){detail}")
         self.code = code
 
 

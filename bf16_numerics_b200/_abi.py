@@ -31,7 +31,7 @@ KERNEL_NAMES = ("fa_fwd_kernel", "fa_bwd_delta_kernel", "fa_bwd_main_kernel", "f
 # every symbol include/fa_b200.h declares
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_workspace_delta_offset",
            "fa_bwd_workspace_dq_offset", "fa_status_string", "fa_device_error", "fa_timing_enable",
-           "fa_timing_read", "fa_bwd_noalloc")
+           "fa_timing_read", "fa_bwd_noalloc", "fa_last_error_string")
 
 
 class FaRowStats(ctypes.Structure):
@@ -59,6 +59,8 @@ def load() -> ctypes.CDLL:
         getattr(lib, name).restype = sz
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_last_error_string.argtypes = []
+    lib.fa_last_error_string.restype = ctypes.c_char_p
     lib.fa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.fa_device_error.restype = i
     lib.fa_timing_enable.argtypes = [i]

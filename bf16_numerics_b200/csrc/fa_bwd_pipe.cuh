@@ -1,0 +1,428 @@
+// Pipelined backward main kernel for head dimension 64.
+//
+// Same mathematics as fa_bwd_main_kernel (see fa_bwd.cuh): one CTA per
+// (batch, head, 128-key block), looping over the query blocks that see the
+// keys, in the transposed orientation (lane = key).  What changes is the
+// schedule, so that the tensor core and the elementwise work overlap:
+//
+//   * S^T is double-buffered in TMEM: the MMA warp issues S^T of query block
+//     i+2 while the elementwise warps work on block i, and dP^T of block i+1
+//     as soon as block i's dS has been consumed.
+//   * Eight elementwise warps (two warpgroups) split the 128 query columns of
+//     a key row: warpgroup h takes columns [64h, 64h+64).  Each writes its
+//     bf16 P^T and dS^T into the first half of the TMEM columns it has just
+//     read (P^T at S^T cols 64h + [0,32), dS^T at dP^T cols 64h + [0,32)), so
+//     no warpgroup ever overwrites a column the other still has to read.
+//   * dQ_i = dS K is issued as two N = 32 products into the other halves of
+//     the consumed S^T buffer (cols 64h + [32,64)), which no later product of
+//     the same iteration touches.
+//   * Four drain warps move the dQ partial from TMEM into a 128B-swizzled
+//     fp32 tile in shared memory and add it to the fp32 accumulator in global
+//     memory with one TMA tensor reduce-add per 32-column half (rows past N
+//     are clipped by the tensor map).  They also prepare the per-query
+//     vectors (lse or m, 1/l, delta) two blocks ahead.
+//
+// TMEM columns: S^T[0] [0,128)  S^T[1] [128,256)  dP^T [256,384)
+//               dV [384,448)  dK [448,512)
+// Warps: 0-3 and 4-7 elementwise (key t = threadIdx % 128), 8-11 drain
+// (query t), 12 TMA producer, 13 MMA issuer / TMEM owner.
+#pragma once
+
+#include "fa_bwd.cuh"
+
+namespace fa {
+
+struct BwdPipeLayout {
+  static constexpr int D = 64, B = 128, TILE = 128 * 64 * 2, NST = 3;
+  static constexpr int K_OFF = 0, V_OFF = TILE, Q_OFF = 2 * TILE;
+  static constexpr int DO_OFF = Q_OFF + NST * TILE;
+  static constexpr int DS_OFF = DO_OFF + NST * TILE;  // dS^T [keys][queries], two 64-query halves
+  static constexpr int DQS_OFF = DS_OFF + 2 * TILE;   // dQ staging: two [128 rows][32 fp32] swizzled boxes
+  static constexpr int VEC_OFF = DQS_OFF + 2 * TILE;  // [2 stages][3][128] fp32
+  static constexpr int BAR_OFF = VEC_OFF + 2 * 3 * 128 * 4;
+  enum {
+    KV_FULL = 0,
+    Q_FULL = 1,
+    Q_EMPTY = Q_FULL + NST,
+    S_FULL = Q_EMPTY + NST,  // [2]
+    P_FULL = S_FULL + 2,     // [2]
+    DP_FULL = P_FULL + 2,
+    DS_FULL,
+    DQ_FULL,                 // [2]
+    DQ_FREE = DQ_FULL + 2,
+    VEC_FULL,                // [2]
+    VEC_EMPTY = VEC_FULL + 2,  // [2]
+    ACC_DONE = VEC_EMPTY + 2,
+    TEARDOWN,
+    NBAR
+  };
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512, DPT_COL = 256, DV_COL = 384, DK_COL = 448;
+  static constexpr int THREADS = 448;
+};
+
+__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int x, int y, int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(448, 1)
+fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+  using L = BwdPipeLayout;
+  constexpr int TILE = L::TILE, NST = L::NST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+  auto bar = [&](int i) { return base + L::BAR_OFF + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  float* vec = reinterpret_cast<float*>(smem + L::VEC_OFF);  // [s][0]: -a, [s][1]: 1/l, [s][2]: delta
+  const BoundedWait wait{abort_flag, 3u};
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = p.BH;
+  const int kblk = blockIdx.x / BH;
+  const int bh = blockIdx.x - kblk * BH;
+  const int i0 = p.causal ? kblk : 0;
+  const int n_it = p.n_blk - i0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::KV_FULL), 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar(L::Q_FULL + s), 1);
+      mbar_init(bar(L::Q_EMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(L::S_FULL + b), 1);
+      mbar_init(bar(L::P_FULL + b), 256);
+      mbar_init(bar(L::DQ_FULL + b), 1);
+      mbar_init(bar(L::VEC_FULL + b), 128);
+      mbar_init(bar(L::VEC_EMPTY + b), 256);
+    }
+    mbar_init(bar(L::DP_FULL), 1);
+    mbar_init(bar(L::DS_FULL), 256);
+    mbar_init(bar(L::DQ_FREE), 128);
+    mbar_init(bar(L::ACC_DONE), 1);
+    mbar_init(bar(L::TEARDOWN), 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 13) {
+    tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 12) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_expect_tx(bar(L::KV_FULL), 2 * TILE);
+      tma_load_3d(base + L::K_OFF, &tm_k, bar(L::KV_FULL), 0, kblk * L::B, bh);
+      tma_load_3d(base + L::V_OFF, &tm_v, bar(L::KV_FULL), 0, kblk * L::B, bh);
+      int issued[NST];
+      for (int s = 0; s < NST; ++s) issued[s] = -1;
+      for (int i = 0; i < n_it; ++i) {
+        const int s = i % NST, use = i / NST;
+        if (use > 0 && !wait(bar(L::Q_EMPTY + s), (use - 1) & 1, 1)) break;
+        const int row0 = (i0 + i) * L::B;
+        mbar_expect_tx(bar(L::Q_FULL + s), 2 * TILE);
+        tma_load_3d(base + L::Q_OFF + s * TILE, &tm_q, bar(L::Q_FULL + s), 0, row0, bh);
+        tma_load_3d(base + L::DO_OFF + s * TILE, &tm_do, bar(L::Q_FULL + s), 0, row0, bh);
+        issued[s] = i;
+      }
+      volatile int never = 0;
+      const BoundedWait drain{&never, 3u};
+      drain(bar(L::KV_FULL), 0, 20);
+      for (int s = 0; s < NST; ++s)
+        if (issued[s] >= 0) drain(bar(L::Q_FULL + s), (issued[s] / NST) & 1, 21);
+    }
+    __syncwarp();
+  } else if (warp == 13) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_SQ = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
+      constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 64, false, true);    // dV, dK
+      constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, 32, true, true);     // dQ halves
+      auto q_tile = [&](int i) { return base + L::Q_OFF + (i % NST) * TILE; };
+      auto do_tile = [&](int i) { return base + L::DO_OFF + (i % NST) * TILE; };
+      auto issue_s = [&](int i) {
+        const uint32_t d_tmem = tmem + 128u * (i & 1);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ss(d_tmem, sdesc_sw128(base + L::K_OFF + ks * 32, 16, 1024), sdesc_sw128(q_tile(i) + ks * 32, 16, 1024),
+                 IDESC_SQ, ks > 0 ? 1u : 0u);
+        tc_commit(bar(L::S_FULL + (i & 1)));
+      };
+      auto issue_dp = [&](int i) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ss(tmem + L::DPT_COL, sdesc_sw128(base + L::V_OFF + ks * 32, 16, 1024),
+                 sdesc_sw128(do_tile(i) + ks * 32, 16, 1024), IDESC_SQ, ks > 0 ? 1u : 0u);
+        tc_commit(bar(L::DP_FULL));
+      };
+      bool ok = wait(bar(L::KV_FULL), 0, 2);
+      if (ok && n_it > 0) {
+        ok = wait(bar(L::Q_FULL + 0), 0, 3);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+          issue_dp(0);
+        }
+      }
+      if (ok && n_it > 1) {
+        ok = wait(bar(L::Q_FULL + 1), 0, 3);
+        if (ok) {
+          tc_fence_after();
+          issue_s(1);
+        }
+      }
+      for (int i = 0; ok && i < n_it; ++i) {
+        const int b = i & 1;
+        if (!wait(bar(L::P_FULL + b), (i >> 1) & 1, 4)) break;
+        tc_fence_after();
+        // dV += P^T dO_i   (K-dim = queries; P^T of half h at S^T cols 64h + [0,32))
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t a = tmem + 128u * b + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4));
+          mma_ts(tmem + L::DV_COL, a, sdesc_sw128(do_tile(i) + ks * 2048, 16384, 1024), IDESC_KV,
+                 (i > 0 || ks > 0) ? 1u : 0u);
+        }
+        if (!wait(bar(L::DS_FULL), i & 1, 5)) break;
+        tc_fence_after();
+        // dK += dS^T Q_i
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t a = tmem + L::DPT_COL + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4));
+          mma_ts(tmem + L::DK_COL, a, sdesc_sw128(q_tile(i) + ks * 2048, 16384, 1024), IDESC_KV,
+                 (i > 0 || ks > 0) ? 1u : 0u);
+        }
+        // dQ_i = dS K, as two 32-column halves into the consumed S^T columns 64h + [32,64)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + 128u * b + 32u + 64u * h, sdesc_sw128(base + L::DS_OFF + ks * 2048, 16384, 1024),
+                   sdesc_sw128(base + L::K_OFF + ks * 2048 + 64 * h, 16384, 1024), IDESC_DQ, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(L::DQ_FULL + b));
+        tc_commit(bar(L::Q_EMPTY + (i % NST)));
+        if (i + 1 < n_it) issue_dp(i + 1);
+        if (i + 2 < n_it) {
+          if (!wait(bar(L::DQ_FREE), i & 1, 6)) break;
+          if (!wait(bar(L::Q_FULL + ((i + 2) % NST)), ((i + 2) / NST) & 1, 7)) break;
+          tc_fence_after();
+          issue_s(i + 2);
+        }
+      }
+      tc_commit(bar(L::ACC_DONE));
+      tc_commit(bar(L::TEARDOWN));
+    }
+    __syncwarp();
+  } else if (warp >= 8) {
+    // --------------------------------------------------------- drain warps
+    const int t = threadIdx.x - 256;  // query within the block == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float scale = p.scale;
+    const size_t vrow0 = static_cast<size_t>(bh) * p.N;
+    auto prep = [&](int i) {
+      const int s = i & 1, q = (i0 + i) * L::B + t;
+      float na = -INFINITY, bb = 0.f, dl = 0.f;
+      if (q < p.N) {
+        const float lse = __ldg(p.lse + vrow0 + q);
+        dl = __ldg(p.delta + vrow0 + q);
+        if (p.mode == 1) {
+          const float m = __ldg(p.row_m + vrow0 + q);
+          na = -m * kLog2e;
+          bb = 1.f / ex2_approx((lse - m) * kLog2e);
+        } else {
+          na = -lse * kLog2e;
+          bb = 1.f;
+        }
+      }
+      vec[(s * 3 + 0) * 128 + t] = na;
+      vec[(s * 3 + 1) * 128 + t] = bb;
+      vec[(s * 3 + 2) * 128 + t] = dl;
+      mbar_arrive(bar(L::VEC_FULL + s));
+    };
+    if (n_it > 0) prep(0);
+    if (n_it > 1) prep(1);
+    if (t == 0) tma_prefetch_desc(&tm_dq);
+    for (int i = 0; i < n_it; ++i) {
+      const int b = i & 1;
+      if (!wait(bar(L::DQ_FULL + b), (i >> 1) & 1, 13)) break;
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld32x2(tmem + lane_base + 128u * b + 32u, tmem + lane_base + 128u * b + 96u, r0, r1);
+      tc_fence_before();
+      mbar_arrive(bar(L::DQ_FREE));
+      if (t == 0) bulk_wait_read_all();  // the previous reduce has finished reading the staging tile
+      named_barrier_sync(2, 128);
+      // row t of each 32-column box, 16-byte chunk c stored at chunk c ^ (t & 7)
+      uint8_t* row0 = smem + L::DQS_OFF + t * 128;
+      uint8_t* row1 = row0 + TILE;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int pc = (c ^ (t & 7)) << 4;
+        *reinterpret_cast<float4*>(row0 + pc) =
+            make_float4(__uint_as_float(r0[4 * c]) * scale, __uint_as_float(r0[4 * c + 1]) * scale,
+                        __uint_as_float(r0[4 * c + 2]) * scale, __uint_as_float(r0[4 * c + 3]) * scale);
+        *reinterpret_cast<float4*>(row1 + pc) =
+            make_float4(__uint_as_float(r1[4 * c]) * scale, __uint_as_float(r1[4 * c + 1]) * scale,
+                        __uint_as_float(r1[4 * c + 2]) * scale, __uint_as_float(r1[4 * c + 3]) * scale);
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(2, 128);
+      if (t == 0) {
+        const int q0 = (i0 + i) * L::B;
+        tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF, 0, q0, bh);
+        tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF + TILE, 32, q0, bh);
+        bulk_commit();
+      }
+      if (i + 2 < n_it) {
+        if (!wait(bar(L::VEC_EMPTY + b), (i >> 1) & 1, 14)) break;
+        prep(i + 2);
+      }
+    }
+    if (t == 0) bulk_wait_all();
+  } else {
+    // ----------------------------------------------- elementwise warps 0..7
+    const int h = warp >> 2;          // query half
+    const int t = threadIdx.x & 127;  // key within the block == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int key = kblk * L::B + t;
+    const float scale = p.scale;
+    const float c_log2 = scale * kLog2e;
+    const uint64_t C2 = f2_pack(c_log2, c_log2);
+    const bool mode1 = p.mode == 1;
+    bool ok = true;
+    for (int i = 0; i < n_it; ++i) {
+      const int b = i & 1;
+      if (!wait(bar(L::VEC_FULL + b), (i >> 1) & 1, 8)) { ok = false; break; }
+      if (!wait(bar(L::S_FULL + b), (i >> 1) & 1, 9)) { ok = false; break; }
+      tc_fence_after();
+      const float* va = vec + (b * 3 + 0) * 128 + 64 * h;
+      const float* vb = vec + (b * 3 + 1) * 128 + 64 * h;
+      const float* vd = vec + (b * 3 + 2) * 128 + 64 * h;
+      const bool diag = p.causal && (i0 + i == kblk);
+      const int qoff = 64 * h;
+      uint64_t p2[32];  // this row's 64 P values (fp32 pairs)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + 128u * b + 64u * h + 32u * c, r);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int ql = 32 * c + 2 * e;
+          const float2 na = *reinterpret_cast<const float2*>(va + ql);
+          const uint64_t y = f2_fma(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), C2,
+                                    f2_pack(na.x, na.y));
+          float y0, y1;
+          f2_unpack(y, y0, y1);
+          float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+          if (mode1) {
+            const float2 bb = *reinterpret_cast<const float2*>(vb + ql);
+            p0 *= bb.x;
+            p1 *= bb.y;
+          }
+          if (diag) {
+            if (t > qoff + ql) p0 = 0.f;
+            if (t > qoff + ql + 1) p1 = 0.f;
+          }
+          p2[16 * c + e] = f2_pack(p0, p1);
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tmem + lane_base + 128u * b + 64u * h + 16u * c, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(L::P_FULL + b));
+      if (!wait(bar(L::DP_FULL), i & 1, 10)) { ok = false; break; }
+      // the dQ product of the previous block has finished reading the dS tile
+      if (i > 0 && !wait(bar(L::DQ_FULL + ((i - 1) & 1)), ((i - 1) >> 1) & 1, 11)) { ok = false; break; }
+      tc_fence_after();
+      uint8_t* ds_row = smem + L::DS_OFF + h * TILE + t * 128;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + L::DPT_COL + 64u * h + 32u * c, r);
+        uint32_t dk_[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int ql = 32 * c + 2 * e;
+          const float2 dl = *reinterpret_cast<const float2*>(vd + ql);
+          const uint64_t ds = f2_mul(p2[16 * c + e], f2_sub(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])),
+                                                            f2_pack(dl.x, dl.y)));
+          float d0, d1;
+          f2_unpack(ds, d0, d1);
+          dk_[e] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tmem + lane_base + L::DPT_COL + 64u * h + 16u * c, dk_);
+        // dS^T row t, queries 64h + 32c + [0,32) = 16-byte chunks 4c..4c+3 of the half tile
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int chunk = 4 * c + j;
+          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (t & 7)) << 4)) =
+              make_uint4(dk_[4 * j], dk_[4 * j + 1], dk_[4 * j + 2], dk_[4 * j + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(L::DS_FULL));
+      mbar_arrive(bar(L::VEC_EMPTY + b));
+    }
+    // ------------------------------------------------------------- epilogue
+    if (ok && wait(bar(L::ACC_DONE), 0, 12)) {
+      tc_fence_after();
+      const bool row_ok = key < p.N;
+      const float f = (h == 0) ? 1.f : scale;  // warpgroup 0 writes dV, warpgroup 1 writes dK * scale
+      __nv_bfloat16* dst = (h == 0 ? p.dv : p.dk) + (static_cast<size_t>(bh) * p.N + key) * 64;
+      uint32_t r0[32], r1[32];
+      const uint32_t col = (h == 0) ? L::DV_COL : L::DK_COL;
+      tmem_ld32x2(tmem + lane_base + col, tmem + lane_base + col + 32, r0, r1);
+      if (row_ok) {
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          uint4 w0, w1;
+          w0.x = pack_bf16x2(__uint_as_float(r0[c + 0]) * f, __uint_as_float(r0[c + 1]) * f);
+          w0.y = pack_bf16x2(__uint_as_float(r0[c + 2]) * f, __uint_as_float(r0[c + 3]) * f);
+          w0.z = pack_bf16x2(__uint_as_float(r0[c + 4]) * f, __uint_as_float(r0[c + 5]) * f);
+          w0.w = pack_bf16x2(__uint_as_float(r0[c + 6]) * f, __uint_as_float(r0[c + 7]) * f);
+          w1.x = pack_bf16x2(__uint_as_float(r1[c + 0]) * f, __uint_as_float(r1[c + 1]) * f);
+          w1.y = pack_bf16x2(__uint_as_float(r1[c + 2]) * f, __uint_as_float(r1[c + 3]) * f);
+          w1.z = pack_bf16x2(__uint_as_float(r1[c + 4]) * f, __uint_as_float(r1[c + 5]) * f);
+          w1.w = pack_bf16x2(__uint_as_float(r1[c + 6]) * f, __uint_as_float(r1[c + 7]) * f);
+          *reinterpret_cast<uint4*>(dst + c) = w0;
+          *reinterpret_cast<uint4*>(dst + 32 + c) = w1;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    volatile int never = 0;
+    const BoundedWait drain{&never, 3u};
+    drain(bar(L::TEARDOWN), 0, 30);
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

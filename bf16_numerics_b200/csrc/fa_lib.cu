@@ -6,12 +6,13 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <vector>
 
 #include "fa_b200.h"
-#include "fa_bwd.cuh"
+#include "fa_bwd_pipe.cuh"
 
 namespace {
 
@@ -48,6 +49,33 @@ bool make_map(CUtensorMap* map, const void* ptr, long long BH, long long N, int 
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// fp32 dQ accumulator [BH, N, 64] -> 3-D tensor map, box 32 (d) x 128 (rows) x 1,
+// 128B swizzle: the target of the pipelined backward's TMA reduce-add.
+bool make_map_dq(CUtensorMap* map, const void* ptr, long long BH, long long N) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {64 * 4, static_cast<cuuint64_t>(N) * 64 * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Last CUDA failure seen by this thread's fa_* call: "<what>: <cudaError name>".
+thread_local char g_last_error[256] = "";
+
+fa_status cuda_fail(const char* what, cudaError_t e) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorName(e));
+  return FA_ERR_CUDA;
+}
+fa_status cuda_fail(const char* what) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s", what);
+  return FA_ERR_CUDA;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -99,7 +127,12 @@ struct LaunchTimer {
 
 template <typename K>
 bool set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    cuda_fail("cudaFuncSetAttribute(max dynamic shared memory)", e);
+    return false;
+  }
+  return true;
 }
 
 bool shape_ok(int B, int H, int N, int d) {
@@ -121,7 +154,8 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
     attr = true;
   }
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D)) return FA_ERR_CUDA;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
+    return cuda_fail("cuTensorMapEncodeTiled (q/k/v)");
   fa::FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -142,7 +176,8 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   LaunchTimer tm(FA_KERNEL_FWD, stream);
   fa::fa_fwd_kernel<D><<<grid, 192, L::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   tm.done();
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail("fa_fwd_kernel launch", e);
 }
 
 int grid_for(long long work, int per_block) {
@@ -157,9 +192,14 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      const float* row_m, void* dq, void* dk, void* dv, uint8_t* ws, int BH, int N, int causal,
                      int mode, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
+  using LP = fa::BwdPipeLayout;
   static bool attr = false;
   if (!attr) {
-    if (!set_smem(fa::fa_bwd_main_kernel<D>, L::SMEM_BYTES)) return FA_ERR_CUDA;
+    if (D == 64) {
+      if (!set_smem(fa::fa_bwd_main_pipe_kernel, LP::SMEM_BYTES)) return FA_ERR_CUDA;
+    } else {
+      if (!set_smem(fa::fa_bwd_main_kernel<D>, L::SMEM_BYTES)) return FA_ERR_CUDA;
+    }
     attr = true;
   }
   const long long rows = static_cast<long long>(BH) * N;
@@ -168,14 +208,15 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D) ||
       !make_map(&mdo, dO, BH, N, D))
-    return FA_ERR_CUDA;
+    return cuda_fail("cuTensorMapEncodeTiled (q/k/v/dO)");
   {
     constexpr int rows_per_block = 8 * (32 / (D / 8));
     LaunchTimer tm(FA_KERNEL_BWD_DELTA, stream);
     fa::fa_bwd_delta_kernel<D><<<grid_for(rows, rows_per_block), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows);
     tm.done();
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("fa_bwd_delta_kernel launch", e);
   }
   {
     fa::BwdParams p{};
@@ -192,10 +233,19 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.mode = mode;
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_blk) * BH);
-    LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
-    fa::fa_bwd_main_kernel<D><<<grid, 320, L::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
-    tm.done();
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (D == 64) {
+      CUtensorMap mdq;
+      if (!make_map_dq(&mdq, dq_acc, BH, N)) return cuda_fail("cuTensorMapEncodeTiled (dQ accumulator)");
+      LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
+      fa::fa_bwd_main_pipe_kernel<<<grid, LP::THREADS, LP::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
+      tm.done();
+    } else {
+      LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
+      fa::fa_bwd_main_kernel<D><<<grid, 320, L::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
+      tm.done();
+    }
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
   }
   {
     const long long n8 = rows * D / 8;
@@ -203,7 +253,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     fa::fa_bwd_dq_convert_kernel<<<grid_for(n8, 256), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
                                                                          n8);
     tm.done();
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("fa_bwd_dq_convert_kernel launch", e);
   }
   return FA_OK;
 }
@@ -287,6 +338,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (d == 64) return launch_bwd<64>(q, k, v, o, dO, lse, row_m, dq, dk, dv, ws, BH, N, causal, softmax_mode, s);
   return launch_bwd<128>(q, k, v, o, dO, lse, row_m, dq, dk, dv, ws, BH, N, causal, softmax_mode, s);
 }
+
+const char* fa_last_error_string(void) { return g_last_error; }
 
 fa_status fa_device_error(unsigned int* code) {
   if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;

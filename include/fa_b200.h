@@ -108,6 +108,11 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
 /* Static description of a status code. */
 const char* fa_status_string(fa_status s);
 
+/* The CUDA failure behind the last FA_ERR_CUDA returned to the calling
+ * thread: the failing step and CUDA's error name (thread-local storage owned
+ * by the library; "" if none yet). */
+const char* fa_last_error_string(void);
+
 /* Synchronises the current device, then reads and clears the device error
  * word that kernels set when a bounded wait ran out.  *code (may be NULL)
  * receives the raw word (kernel id << 24 | wait site << 16 | block).
