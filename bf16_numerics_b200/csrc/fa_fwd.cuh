@@ -17,9 +17,17 @@
 //              rescale and the epilogue;
 //   warp  4    TMA producer (Q once, K/V through a 2-stage ring);
 //   warp  5    MMA issuer (one thread) and TMEM owner.
-// TMEM columns: S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384)
-//               O [384, 384+D).  P_bar is stored back into TMEM as packed
-// bf16 pairs and fed to the P V product as the A operand straight from TMEM.
+// TMEM columns: S [0,128)  P_bar [128,192) (bf16 pairs)  O [192, 192+D).
+// With d = 64 that is 256 columns and two CTAs share an SM, so eight softmax
+// warps hide each other's latency.  S is single-buffered: the softmax warps
+// copy it to registers first and release it, so the next tile's Q K^T runs on
+// the tensor core while they work; P_bar is fed to the P V product as the A
+// operand straight from TMEM.
+//
+// For d = 64 the scale 1/8 is a power of two, so comparisons (max, ties) are
+// taken on the raw fp32 accumulator: x == y <=> x/8 == y/8 and rm = max/8
+// exactly.  For d = 128 the scores are scaled first (fp32 multiply), because
+// two raw values one ulp apart can round to the same scaled value.
 #pragma once
 
 #include "fa_ptx.cuh"
@@ -50,21 +58,20 @@ struct FwdLayout {
   static constexpr int V_OFF = K_OFF + 2 * TILE;
   static constexpr int BAR_OFF = V_OFF + 2 * TILE;
   // barrier indices
-  enum { Q_FULL = 0, K_FULL = 1, V_FULL = 3, KV_EMPTY = 5, S_FULL = 7, S_FREE = 9, P_FULL = 11,
-         O_READY = 13, TEARDOWN = 14, NBAR = 15 };
+  enum { Q_FULL = 0, K_FULL = 1, V_FULL = 3, KV_EMPTY = 5, S_FULL = 7, S_FREE, P_FULL, O_READY, TEARDOWN, NBAR };
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base (4B), abort flag (4B)
-  static constexpr int USED = MISC_OFF + 16;
-  // force one CTA per SM: each CTA owns all 512 TMEM columns
-  static constexpr int SMEM_BYTES = (USED + 1024 > 120 * 1024 ? USED + 1024 : 120 * 1024);
-  static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t S_COL0 = 0, P_COL0 = 256, O_COL = 384;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr uint32_t S_COL = 0, P_COL = 128, O_COL = 192;
+  static constexpr uint32_t TMEM_COLS = (O_COL + D <= 256) ? 256 : 512;
+  static constexpr int CTAS_PER_SM = (TMEM_COLS == 256) ? 2 : 1;
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, FwdLayout<D>::CTAS_PER_SM)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using L = FwdLayout<D>;
+  constexpr bool kRawCompare = (D == 64);  // scale is exactly 1/8
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;  // 1024-byte aligned for the 128B swizzle
@@ -88,10 +95,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_init(bar(L::K_FULL + s), 1);
       mbar_init(bar(L::V_FULL + s), 1);
       mbar_init(bar(L::KV_EMPTY + s), 1);
-      mbar_init(bar(L::S_FULL + s), 1);
-      mbar_init(bar(L::S_FREE + s), 128);
-      mbar_init(bar(L::P_FULL + s), 128);
     }
+    mbar_init(bar(L::S_FULL), 1);
+    mbar_init(bar(L::S_FREE), 128);
+    mbar_init(bar(L::P_FULL), 128);
     mbar_init(bar(L::O_READY), 1);
     mbar_init(bar(L::TEARDOWN), 1);
     *abort_flag = 0;
@@ -144,37 +151,40 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
-      bool ok = wait(bar(L::Q_FULL), 0, 2);
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {
-          const int s = j & 1;
-          if (!wait(bar(L::K_FULL + s), (j >> 1) & 1, 3)) break;
-          if (j >= 2 && !wait(bar(L::S_FREE + s), ((j >> 1) - 1) & 1, 4)) break;
-          tc_fence_after();
-          const uint32_t d_tmem = tmem + L::S_COL0 + 128u * s;
+      auto issue_s = [&](int j) {
+        const int s = j & 1;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t koff = (ks >> 2) * L::HALF + (ks & 3) * 32;
-            const uint64_t a = sdesc_sw128(base + L::Q_OFF + koff, 16, 1024);
-            const uint64_t b = sdesc_sw128(base + L::K_OFF + s * L::TILE + koff, 16, 1024);
-            mma_ss(d_tmem, a, b, IDESC_S, ks > 0 ? 1u : 0u);
-          }
-          tc_commit(bar(L::S_FULL + s));
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t koff = (ks >> 2) * L::HALF + (ks & 3) * 32;
+          mma_ss(tmem + L::S_COL, sdesc_sw128(base + L::Q_OFF + koff, 16, 1024),
+                 sdesc_sw128(base + L::K_OFF + s * L::TILE + koff, 16, 1024), IDESC_S, ks > 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          const int jj = j - 1, s = jj & 1;
-          if (!wait(bar(L::P_FULL + s), (jj >> 1) & 1, 5)) break;
-          if (!wait(bar(L::V_FULL + s), (jj >> 1) & 1, 6)) break;
+        tc_commit(bar(L::S_FULL));
+      };
+      bool ok = wait(bar(L::Q_FULL), 0, 2) && wait(bar(L::K_FULL), 0, 3);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int s = j & 1;
+        // S of the next tile as soon as the softmax warps have copied S_j out
+        if (j + 1 < nkv) {
+          if (!wait(bar(L::S_FREE), j & 1, 4)) break;
+          if (!wait(bar(L::K_FULL + ((j + 1) & 1)), ((j + 1) >> 1) & 1, 3)) break;
           tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < L::BN / 16; ++ks) {
-            const uint32_t a_tmem = tmem + L::P_COL0 + 64u * s + 8u * ks;
-            const uint64_t b = sdesc_sw128(base + L::V_OFF + s * L::TILE + ks * 2048, L::HALF, 1024);
-            mma_ts(tmem + L::O_COL, a_tmem, b, IDESC_O, (jj > 0 || ks > 0) ? 1u : 0u);
-          }
-          tc_commit(bar(L::O_READY));
-          tc_commit(bar(L::KV_EMPTY + s));
+          issue_s(j + 1);
         }
+        if (!wait(bar(L::P_FULL), j & 1, 5)) break;
+        if (!wait(bar(L::V_FULL + s), (j >> 1) & 1, 6)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < L::BN / 16; ++ks) {
+          const uint64_t b = sdesc_sw128(base + L::V_OFF + s * L::TILE + ks * 2048, L::HALF, 1024);
+          mma_ts(tmem + L::O_COL, tmem + L::P_COL + 8u * ks, b, IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        tc_commit(bar(L::O_READY));
+        tc_commit(bar(L::KV_EMPTY + s));
       }
       tc_commit(bar(L::TEARDOWN));
     }
@@ -184,18 +194,24 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int t = threadIdx.x;  // row within the tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int q_row = qblk * L::BM + t;
-    const float scale = p.scale, beta = p.beta;
-    float rm = -INFINITY, m_run = -INFINITY, l = 0.f;
+    // compare domain: raw accumulator (d = 64) or scaled scores (d = 128)
+    const float cmp_scale = kRawCompare ? 1.f : p.scale;        // x = acc * cmp_scale
+    const float to_s = kRawCompare ? p.scale : 1.f;             // S = x * to_s (exact)
+    const float exp_c = (kRawCompare ? p.scale : 1.f) * kLog2e; // exp2 argument per unit of x
+    const uint64_t EXPC2 = f2_pack(exp_c, exp_c);
+    const float beta = p.beta;
+    float rm_x = -INFINITY;  // running row max, x domain
+    float m_run = -INFINITY; // shift in force, S domain
+    float l = 0.f;
     int rs = 0;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int s = j & 1;
-      if (!wait(bar(L::S_FULL + s), (j >> 1) & 1, 7)) { ok = false; break; }
+      if (!wait(bar(L::S_FULL), j & 1, 7)) { ok = false; break; }
       tc_fence_after();
       float x[128];
       {
         uint32_t r0[32], r1[32];
-        const uint32_t sa = tmem + lane_base + L::S_COL0 + 128u * s;
+        const uint32_t sa = tmem + lane_base + L::S_COL;
         tmem_ld32x2(sa, sa + 32, r0, r1);
 #pragma unroll
         for (int c = 0; c < 32; ++c) { x[c] = __uint_as_float(r0[c]); x[32 + c] = __uint_as_float(r1[c]); }
@@ -204,28 +220,50 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int c = 0; c < 32; ++c) { x[64 + c] = __uint_as_float(r0[c]); x[96 + c] = __uint_as_float(r1[c]); }
       }
       tc_fence_before();
-      mbar_arrive(bar(L::S_FREE + s));
-      // scores in the S domain, masked entries -inf
+      mbar_arrive(bar(L::S_FREE));
+      // mask (diagonal tile / ragged tail) and tile max, eight partial maxima
       const int kv0 = j * L::BN;
       const bool diag = p.causal && (j == qblk);
       const int lim_causal = diag ? t : (L::BN - 1);
       const int lim_len = p.N - 1 - kv0;
       const int lim = lim_causal < lim_len ? lim_causal : lim_len;
-      float tmax = -INFINITY;
+      const bool masked = (lim < L::BN - 1);
+      float pm[8];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float v = (c <= lim) ? x[c] * scale : -INFINITY;
-        x[c] = v;
-        tmax = fmaxf(tmax, v);
+      for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+      if (masked) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const float v = (c <= lim) ? x[c] * cmp_scale : -INFINITY;
+          x[c] = v;
+          pm[c & 7] = fmaxf(pm[c & 7], v);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          if (!kRawCompare) x[c] *= cmp_scale;
+          pm[c & 7] = fmaxf(pm[c & 7], x[c]);
+        }
       }
-      int tcnt = 0;
+      const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      // tie count: only rows whose tile max reaches the running max need it
+      if (__any_sync(0xffffffffu, tmax >= rm_x)) {
+        int cnt[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int c = 0; c < 128; ++c) tcnt += (x[c] == tmax) ? 1 : 0;
-      if (tmax > rm) { rm = tmax; rs = tcnt; }
-      else if (tmax == rm) { rs += tcnt; }
-      float m_new = rm;
-      if (p.mode == 1 && rs > 1) m_new = (rm > 0.f) ? beta * rm : ((rm < 0.f) ? 0.f : beta - 1.f);
-      // O and P[s] are free once the previous P V product has completed
+        for (int c = 0; c < 128; ++c) cnt[c & 3] += (x[c] == tmax) ? 1 : 0;
+        const int tc = (cnt[0] + cnt[1]) + (cnt[2] + cnt[3]);
+        if (tmax > rm_x) {
+          rm_x = tmax;
+          rs = tc;
+        } else if (tmax == rm_x) {
+          rs += tc;
+        }
+      }
+      const float rm_s = rm_x * to_s;
+      float m_new = rm_s;
+      if (p.mode == 1 && rs > 1) m_new = (rm_s > 0.f) ? beta * rm_s : ((rm_s < 0.f) ? 0.f : beta - 1.f);
+      // P and O are free once the previous P V product has completed
       if (j > 0) {
         if (!wait(bar(L::O_READY), (j - 1) & 1, 8)) { ok = false; break; }
         tc_fence_after();
@@ -236,39 +274,49 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           l *= alpha;
         }
         if (__any_sync(0xffffffffu, changed)) {
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t r[32];
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            uint32_t r[16];
             const uint32_t oa = tmem + lane_base + L::O_COL + c0;
-            tmem_ld32(oa, r);
+            tmem_ld16(oa, r);
+            uint32_t w[16];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-            tmem_st32(oa, r);
+            for (int c = 0; c < 16; ++c) w[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+            tmem_st16(oa, w);
           }
         }
       }
       m_run = m_new;
-      // P_bar = exp(S - m), rowsum in fp32, bf16 operand into TMEM
-      float rsum = 0.f;
+      // P_bar = exp2(x * exp_c - m * log2e); row sum in fp32 (four pair accumulators)
+      const float nm = -m_new * kLog2e;
+      const uint64_t NM2 = f2_pack(nm, nm);
+      uint64_t sum2[2] = {0ull, 0ull};
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t pk[16];
+      for (int c0 = 0; c0 < 128; c0 += 16) {
+        uint32_t pk[8];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float e0 = ex2_approx((x[c0 + c] - m_new) * kLog2e);
-          const float e1 = ex2_approx((x[c0 + c + 1] - m_new) * kLog2e);
-          rsum += e0 + e1;
+        for (int c = 0; c < 16; c += 2) {
+          const uint64_t y = f2_fma(f2_pack(x[c0 + c], x[c0 + c + 1]), EXPC2, NM2);
+          float y0, y1;
+          f2_unpack(y, y0, y1);
+          const float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
+          sum2[(c >> 1) & 1] = f2_add(sum2[(c >> 1) & 1], f2_pack(e0, e1));
           pk[c >> 1] = pack_bf16x2(e0, e1);
         }
-        tmem_st16(tmem + lane_base + L::P_COL0 + 64u * s + (c0 >> 1), pk);
+        tmem_st8(tmem + lane_base + L::P_COL + (c0 >> 1), pk);
       }
-      l += rsum;
+      {
+        const uint64_t s01 = f2_add(sum2[0], sum2[1]);
+        float a, b;
+        f2_unpack(s01, a, b);
+        l += a + b;
+      }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(L::P_FULL + s));
+      mbar_arrive(bar(L::P_FULL));
     }
     // ------------------------------------------------------------- epilogue
-    if (ok && wait(bar(L::O_READY), (nkv - 1) & 1, 9)) {
+    if (ok && nkv > 0 && wait(bar(L::O_READY), (nkv - 1) & 1, 9)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool row_ok = q_row < p.N;
@@ -291,11 +339,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       if (row_ok) {
         const size_t ri = static_cast<size_t>(bh) * p.N + q_row;
+        const float rm_s = rm_x * to_s;
         p.lse[ri] = m_run + logf(l);
-        if (p.st_rm) p.st_rm[ri] = rm;
+        if (p.st_rm) p.st_rm[ri] = rm_s;
         if (p.st_rs) p.st_rs[ri] = rs;
         if (p.st_m) p.st_m[ri] = m_run;
-        if (p.st_pbar_max) p.st_pbar_max[ri] = ex2_approx((rm - m_run) * kLog2e);
+        if (p.st_pbar_max) p.st_pbar_max[ri] = ex2_approx((rm_s - m_run) * kLog2e);
       }
     }
   }
