@@ -37,8 +37,9 @@ namespace fa {
 
 // ------------------------------------------------------------------ delta
 // delta[r] = sum_c dO[r,c] * O[r,c] in fp32; also clears the dQ accumulator
-// row.  Memory bound: each row of O and dO is read once with 16-byte loads,
-// LPR lanes per row.
+// row.
+// Memory bound: each row of O and dO is read once with 16-byte loads, LPR
+// lanes per row.
 template <int D>
 __global__ void __launch_bounds__(256)
 fa_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,

@@ -9,13 +9,14 @@
 //     i+2 while the elementwise warps work on block i, and dP^T of block i+1
 //     as soon as block i's dS has been consumed.
 //   * Eight elementwise warps (two warpgroups) split the 128 query columns of
-//     a key row: warpgroup h takes columns [64h, 64h+64).  Each writes its
-//     bf16 P^T and dS^T into the first half of the TMEM columns it has just
-//     read (P^T at S^T cols 64h + [0,32), dS^T at dP^T cols 64h + [0,32)), so
-//     no warpgroup ever overwrites a column the other still has to read.
-//   * dQ_i = dS K is issued as two N = 32 products into the other halves of
-//     the consumed S^T buffer (cols 64h + [32,64)), which no later product of
-//     the same iteration touches.
+//     a key row: warpgroup h takes columns [64h, 64h+64).  Both copy their S^T
+//     columns to registers and meet at a named barrier; then warpgroup h
+//     writes its bf16 P^T into S^T cols [32h, 32h+32), so P^T occupies
+//     [0,64) and [64,128) is free for dQ.  dS^T goes into the first half of
+//     the dP^T columns each warpgroup has just read (64h + [0,32)), which
+//     needs no barrier.
+//   * dQ_i = dS K is one N = 64 product into S^T cols [64,128) of the same
+//     buffer, which no later product of the iteration touches.
 //   * Four drain warps move the dQ partial from TMEM into a 128B-swizzled
 //     fp32 tile in shared memory and add it to the fp32 accumulator in global
 //     memory with one TMA tensor reduce-add per 32-column half (rows past N
@@ -73,7 +74,8 @@ __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src
 __global__ void __launch_bounds__(448, 1)
 fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                        const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+                        const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+                        const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   using L = BwdPipeLayout;
   constexpr int TILE = L::TILE, NST = L::NST;
   extern __shared__ uint8_t smem_raw[];
@@ -94,6 +96,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   const int n_it = p.n_blk - i0;
 
   if (threadIdx.x == 0) {
+    FA_TRACE_POINT(0);
     mbar_init(bar(L::KV_FULL), 1);
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar(L::Q_FULL + s), 1);
@@ -122,6 +125,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) FA_TRACE_POINT(1);
 
   if (warp == 12) {
     // ------------------------------------------------------------ TMA producer
@@ -156,7 +160,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     if (lane == 0) {
       constexpr uint32_t IDESC_SQ = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 64, false, true);    // dV, dK
-      constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, 32, true, true);     // dQ halves
+      constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, 64, true, true);     // dQ
       auto q_tile = [&](int i) { return base + L::Q_OFF + (i % NST) * TILE; };
       auto do_tile = [&](int i) { return base + L::DO_OFF + (i % NST) * TILE; };
       auto issue_s = [&](int i) {
@@ -193,15 +197,17 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       for (int i = 0; ok && i < n_it; ++i) {
         const int b = i & 1;
         if (!wait(bar(L::P_FULL + b), (i >> 1) & 1, 4)) break;
+        FA_TRACE_POINT(10);
         tc_fence_after();
-        // dV += P^T dO_i   (K-dim = queries; P^T of half h at S^T cols 64h + [0,32))
+        // dV += P^T dO_i   (K-dim = queries; P^T at S^T cols [0,64))
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t a = tmem + 128u * b + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4));
+          const uint32_t a = tmem + 128u * b + 8u * ks;
           mma_ts(tmem + L::DV_COL, a, sdesc_sw128(do_tile(i) + ks * 2048, 16384, 1024), IDESC_KV,
                  (i > 0 || ks > 0) ? 1u : 0u);
         }
         if (!wait(bar(L::DS_FULL), i & 1, 5)) break;
+        FA_TRACE_POINT(11);
         tc_fence_after();
         // dK += dS^T Q_i
 #pragma unroll
@@ -210,19 +216,18 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           mma_ts(tmem + L::DK_COL, a, sdesc_sw128(q_tile(i) + ks * 2048, 16384, 1024), IDESC_KV,
                  (i > 0 || ks > 0) ? 1u : 0u);
         }
-        // dQ_i = dS K, as two 32-column halves into the consumed S^T columns 64h + [32,64)
+        // dQ_i = dS K into S^T cols [64,128) of the same buffer
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + 128u * b + 32u + 64u * h, sdesc_sw128(base + L::DS_OFF + ks * 2048, 16384, 1024),
-                   sdesc_sw128(base + L::K_OFF + ks * 2048 + 64 * h, 16384, 1024), IDESC_DQ, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tmem + 128u * b + 64u, sdesc_sw128(base + L::DS_OFF + ks * 2048, 16384, 1024),
+                 sdesc_sw128(base + L::K_OFF + ks * 2048, 16384, 1024), IDESC_DQ, ks > 0 ? 1u : 0u);
         tc_commit(bar(L::DQ_FULL + b));
         tc_commit(bar(L::Q_EMPTY + (i % NST)));
         if (i + 1 < n_it) issue_dp(i + 1);
+        FA_TRACE_POINT(12);
         if (i + 2 < n_it) {
           if (!wait(bar(L::DQ_FREE), i & 1, 6)) break;
+          FA_TRACE_POINT(13);
           if (!wait(bar(L::Q_FULL + ((i + 2) % NST)), ((i + 2) / NST) & 1, 7)) break;
           tc_fence_after();
           issue_s(i + 2);
@@ -238,18 +243,28 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float scale = p.scale;
     const size_t vrow0 = static_cast<size_t>(bh) * p.N;
-    auto prep = [&](int i) {
+    // per-query vectors of block i: global loads first (prefetch), smem later
+    struct Vec3 { float lse, m, dl; };
+    auto load_vec = [&](int i) {
+      Vec3 v{0.f, 0.f, 0.f};
+      const int q = (i0 + i) * L::B + t;
+      if (i < n_it && q < p.N) {
+        v.lse = __ldg(p.lse + vrow0 + q);
+        v.dl = __ldg(p.delta + vrow0 + q);
+        v.m = (p.mode == 1) ? __ldg(p.row_m + vrow0 + q) : 0.f;
+      }
+      return v;
+    };
+    auto publish_vec = [&](int i, const Vec3& v) {
       const int s = i & 1, q = (i0 + i) * L::B + t;
       float na = -INFINITY, bb = 0.f, dl = 0.f;
       if (q < p.N) {
-        const float lse = __ldg(p.lse + vrow0 + q);
-        dl = __ldg(p.delta + vrow0 + q);
+        dl = v.dl;
         if (p.mode == 1) {
-          const float m = __ldg(p.row_m + vrow0 + q);
-          na = -m * kLog2e;
-          bb = 1.f / ex2_approx((lse - m) * kLog2e);
+          na = -v.m * kLog2e;
+          bb = 1.f / ex2_approx((v.lse - v.m) * kLog2e);
         } else {
-          na = -lse * kLog2e;
+          na = -v.lse * kLog2e;
           bb = 1.f;
         }
       }
@@ -258,15 +273,17 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       vec[(s * 3 + 2) * 128 + t] = dl;
       mbar_arrive(bar(L::VEC_FULL + s));
     };
-    if (n_it > 0) prep(0);
-    if (n_it > 1) prep(1);
+    if (n_it > 0) publish_vec(0, load_vec(0));
+    if (n_it > 1) publish_vec(1, load_vec(1));
+    Vec3 next = load_vec(2);
     if (t == 0) tma_prefetch_desc(&tm_dq);
     for (int i = 0; i < n_it; ++i) {
       const int b = i & 1;
       if (!wait(bar(L::DQ_FULL + b), (i >> 1) & 1, 13)) break;
+      if (t == 0) FA_TRACE_POINT(30);
       tc_fence_after();
       uint32_t r0[32], r1[32];
-      tmem_ld32x2(tmem + lane_base + 128u * b + 32u, tmem + lane_base + 128u * b + 96u, r0, r1);
+      tmem_ld32x2(tmem + lane_base + 128u * b + 64u, tmem + lane_base + 128u * b + 96u, r0, r1);
       tc_fence_before();
       mbar_arrive(bar(L::DQ_FREE));
       if (t == 0) bulk_wait_read_all();  // the previous reduce has finished reading the staging tile
@@ -291,10 +308,12 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF, 0, q0, bh);
         tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF + TILE, 32, q0, bh);
         bulk_commit();
+        FA_TRACE_POINT(31);
       }
       if (i + 2 < n_it) {
         if (!wait(bar(L::VEC_EMPTY + b), (i >> 1) & 1, 14)) break;
-        prep(i + 2);
+        publish_vec(i + 2, next);
+        next = load_vec(i + 3);
       }
     }
     if (t == 0) bulk_wait_all();
@@ -313,6 +332,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       const int b = i & 1;
       if (!wait(bar(L::VEC_FULL + b), (i >> 1) & 1, 8)) { ok = false; break; }
       if (!wait(bar(L::S_FULL + b), (i >> 1) & 1, 9)) { ok = false; break; }
+      if (threadIdx.x == 0) FA_TRACE_POINT(20);
       tc_fence_after();
       const float* va = vec + (b * 3 + 0) * 128 + 64 * h;
       const float* vb = vec + (b * 3 + 1) * 128 + 64 * h;
@@ -320,62 +340,86 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       const bool diag = p.causal && (i0 + i == kblk);
       const int qoff = 64 * h;
       uint64_t p2[32];  // this row's 64 P values (fp32 pairs)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + 128u * b + 64u * h + 32u * c, r);
-        uint32_t pk[16];
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32x2(tmem + lane_base + 128u * b + 64u * h, tmem + lane_base + 128u * b + 64u * h + 32u, r0, r1);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int ql = 32 * c + 2 * e;
-          const float2 na = *reinterpret_cast<const float2*>(va + ql);
-          const uint64_t y = f2_fma(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), C2,
-                                    f2_pack(na.x, na.y));
-          float y0, y1;
-          f2_unpack(y, y0, y1);
-          float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+          p2[e] = f2_pack(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
+          p2[16 + e] = f2_pack(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+        }
+      }
+      // both warpgroups hold their S^T columns: P^T may now overwrite [0,64)
+      named_barrier_sync(1, 256);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          const int pi = 8 * c + e, ql = 2 * pi;
+          const float4 na = *reinterpret_cast<const float4*>(va + ql);
+          const uint64_t y0 = f2_fma(p2[pi], C2, f2_pack(na.x, na.y));
+          const uint64_t y1 = f2_fma(p2[pi + 1], C2, f2_pack(na.z, na.w));
+          float a0, a1, a2, a3;
+          f2_unpack(y0, a0, a1);
+          f2_unpack(y1, a2, a3);
+          float p0 = ex2_approx(a0), p1 = ex2_approx(a1), p2v = ex2_approx(a2), p3 = ex2_approx(a3);
           if (mode1) {
-            const float2 bb = *reinterpret_cast<const float2*>(vb + ql);
+            const float4 bb = *reinterpret_cast<const float4*>(vb + ql);
             p0 *= bb.x;
             p1 *= bb.y;
+            p2v *= bb.z;
+            p3 *= bb.w;
           }
           if (diag) {
-            if (t > qoff + ql) p0 = 0.f;
-            if (t > qoff + ql + 1) p1 = 0.f;
+            const int qg = qoff + ql;
+            if (t > qg) p0 = 0.f;
+            if (t > qg + 1) p1 = 0.f;
+            if (t > qg + 2) p2v = 0.f;
+            if (t > qg + 3) p3 = 0.f;
           }
-          p2[16 * c + e] = f2_pack(p0, p1);
+          p2[pi] = f2_pack(p0, p1);
+          p2[pi + 1] = f2_pack(p2v, p3);
           pk[e] = pack_bf16x2(p0, p1);
+          pk[e + 1] = pack_bf16x2(p2v, p3);
         }
-        tmem_st16(tmem + lane_base + 128u * b + 64u * h + 16u * c, pk);
+        tmem_st8(tmem + lane_base + 128u * b + 32u * h + 8u * c, pk);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::P_FULL + b));
+      if (threadIdx.x == 0) FA_TRACE_POINT(21);
       if (!wait(bar(L::DP_FULL), i & 1, 10)) { ok = false; break; }
+      if (threadIdx.x == 0) FA_TRACE_POINT(22);
       // the dQ product of the previous block has finished reading the dS tile
       if (i > 0 && !wait(bar(L::DQ_FULL + ((i - 1) & 1)), ((i - 1) >> 1) & 1, 11)) { ok = false; break; }
       tc_fence_after();
       uint8_t* ds_row = smem + L::DS_OFF + h * TILE + t * 128;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + L::DPT_COL + 64u * h + 32u * c, r);
-        uint32_t dk_[16];
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[16];
+        tmem_ld16(tmem + lane_base + L::DPT_COL + 64u * h + 16u * c, r);
+        uint32_t dk_[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int ql = 32 * c + 2 * e;
-          const float2 dl = *reinterpret_cast<const float2*>(vd + ql);
-          const uint64_t ds = f2_mul(p2[16 * c + e], f2_sub(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])),
-                                                            f2_pack(dl.x, dl.y)));
-          float d0, d1;
-          f2_unpack(ds, d0, d1);
+        for (int e = 0; e < 8; e += 2) {
+          const int pi = 8 * c + e, ql = 2 * pi;
+          const float4 dl = *reinterpret_cast<const float4*>(vd + ql);
+          const uint64_t ds0 = f2_mul(p2[pi], f2_sub(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])),
+                                                     f2_pack(dl.x, dl.y)));
+          const uint64_t ds1 = f2_mul(p2[pi + 1], f2_sub(f2_pack(__uint_as_float(r[2 * e + 2]), __uint_as_float(r[2 * e + 3])),
+                                                         f2_pack(dl.z, dl.w)));
+          float d0, d1, d2, d3;
+          f2_unpack(ds0, d0, d1);
+          f2_unpack(ds1, d2, d3);
           dk_[e] = pack_bf16x2(d0, d1);
+          dk_[e + 1] = pack_bf16x2(d2, d3);
         }
-        tmem_st16(tmem + lane_base + L::DPT_COL + 64u * h + 16u * c, dk_);
-        // dS^T row t, queries 64h + 32c + [0,32) = 16-byte chunks 4c..4c+3 of the half tile
+        // dS^T into the dP^T columns this warpgroup has read: 64h + [0,32)
+        tmem_st8(tmem + lane_base + L::DPT_COL + 64u * h + 8u * c, dk_);
+        // dS^T row t, queries 64h + 16c + [0,16) = 16-byte chunks 2c, 2c+1 of the half tile
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int chunk = 4 * c + j;
+        for (int j = 0; j < 2; ++j) {
+          const int chunk = 2 * c + j;
           *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (t & 7)) << 4)) =
               make_uint4(dk_[4 * j], dk_[4 * j + 1], dk_[4 * j + 2], dk_[4 * j + 3]);
         }
@@ -385,37 +429,41 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       tc_fence_before();
       mbar_arrive(bar(L::DS_FULL));
       mbar_arrive(bar(L::VEC_EMPTY + b));
+      if (threadIdx.x == 0) FA_TRACE_POINT(24);
     }
     // ------------------------------------------------------------- epilogue
+    // warpgroup 0 writes dV, warpgroup 1 writes dK * scale: TMEM -> bf16 rows
+    // in a 128B-swizzled tile (the dS tile, free once every product is done)
+    // -> one TMA tensor store per warpgroup (rows past N are clipped).
     if (ok && wait(bar(L::ACC_DONE), 0, 12)) {
       tc_fence_after();
-      const bool row_ok = key < p.N;
-      const float f = (h == 0) ? 1.f : scale;  // warpgroup 0 writes dV, warpgroup 1 writes dK * scale
-      __nv_bfloat16* dst = (h == 0 ? p.dv : p.dk) + (static_cast<size_t>(bh) * p.N + key) * 64;
-      uint32_t r0[32], r1[32];
+      const float f = (h == 0) ? 1.f : scale;
       const uint32_t col = (h == 0) ? L::DV_COL : L::DK_COL;
+      uint32_t r0[32], r1[32];
       tmem_ld32x2(tmem + lane_base + col, tmem + lane_base + col + 32, r0, r1);
-      if (row_ok) {
+      uint32_t w[32];
 #pragma unroll
-        for (int c = 0; c < 32; c += 8) {
-          uint4 w0, w1;
-          w0.x = pack_bf16x2(__uint_as_float(r0[c + 0]) * f, __uint_as_float(r0[c + 1]) * f);
-          w0.y = pack_bf16x2(__uint_as_float(r0[c + 2]) * f, __uint_as_float(r0[c + 3]) * f);
-          w0.z = pack_bf16x2(__uint_as_float(r0[c + 4]) * f, __uint_as_float(r0[c + 5]) * f);
-          w0.w = pack_bf16x2(__uint_as_float(r0[c + 6]) * f, __uint_as_float(r0[c + 7]) * f);
-          w1.x = pack_bf16x2(__uint_as_float(r1[c + 0]) * f, __uint_as_float(r1[c + 1]) * f);
-          w1.y = pack_bf16x2(__uint_as_float(r1[c + 2]) * f, __uint_as_float(r1[c + 3]) * f);
-          w1.z = pack_bf16x2(__uint_as_float(r1[c + 4]) * f, __uint_as_float(r1[c + 5]) * f);
-          w1.w = pack_bf16x2(__uint_as_float(r1[c + 6]) * f, __uint_as_float(r1[c + 7]) * f);
-          *reinterpret_cast<uint4*>(dst + c) = w0;
-          *reinterpret_cast<uint4*>(dst + 32 + c) = w1;
-        }
+      for (int c = 0; c < 16; ++c) {
+        w[c] = pack_bf16x2(__uint_as_float(r0[2 * c]) * f, __uint_as_float(r0[2 * c + 1]) * f);
+        w[16 + c] = pack_bf16x2(__uint_as_float(r1[2 * c]) * f, __uint_as_float(r1[2 * c + 1]) * f);
+      }
+      uint8_t* tile = smem + L::DS_OFF + h * TILE;
+      st_row_sw128(tile, t, w);
+      fence_proxy_async_smem();
+      named_barrier_sync(3 + h, 128);
+      if (t == 0) {
+        tma_store_3d(h == 0 ? static_cast<const void*>(&tm_dv) : static_cast<const void*>(&tm_dk),
+                     base + L::DS_OFF + h * TILE, 0, kblk * L::B, bh);
+        bulk_commit();
+        bulk_wait_all();
       }
     }
+    (void)key;
   }
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) FA_TRACE_POINT(2);
   if (warp == 13) {
     tc_fence_after();
     volatile int never = 0;

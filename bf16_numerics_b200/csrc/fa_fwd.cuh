@@ -69,7 +69,8 @@ struct FwdLayout {
 template <int D>
 __global__ void __launch_bounds__(192, FwdLayout<D>::CTAS_PER_SM)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+              const FwdParams p) {
   using L = FwdLayout<D>;
   constexpr bool kRawCompare = (D == 64);  // scale is exactly 1/8
   extern __shared__ uint8_t smem_raw[];
@@ -320,22 +321,26 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool row_ok = q_row < p.N;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + q_row) * D;
+      // O rows -> bf16 in 128B-swizzled 64-column boxes (the K stages, free
+      // once the last P V product has completed) -> TMA tensor store
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + L::O_COL + c0, r);
-        if (row_ok) {
+      for (int h = 0; h < D / 64; ++h) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32x2(tmem + lane_base + L::O_COL + 64 * h, tmem + lane_base + L::O_COL + 64 * h + 32, r0, r1);
+        uint32_t w[32];
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(r[c + 0]) * inv_l, __uint_as_float(r[c + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(r[c + 2]) * inv_l, __uint_as_float(r[c + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(r[c + 4]) * inv_l, __uint_as_float(r[c + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(r[c + 6]) * inv_l, __uint_as_float(r[c + 7]) * inv_l);
-            *reinterpret_cast<uint4*>(orow + c0 + c) = w;
-          }
+        for (int c = 0; c < 16; ++c) {
+          w[c] = pack_bf16x2(__uint_as_float(r0[2 * c]) * inv_l, __uint_as_float(r0[2 * c + 1]) * inv_l);
+          w[16 + c] = pack_bf16x2(__uint_as_float(r1[2 * c]) * inv_l, __uint_as_float(r1[2 * c + 1]) * inv_l);
         }
+        st_row_sw128(smem + L::K_OFF + h * L::HALF, t, w);
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(1, 128);
+      if (t == 0) {
+        for (int h = 0; h < D / 64; ++h) tma_store_3d(&tm_o, base + L::K_OFF + h * L::HALF, 64 * h, qblk * L::BM, bh);
+        bulk_commit();
+        bulk_wait_all();
       }
       if (row_ok) {
         const size_t ri = static_cast<size_t>(bh) * p.N + q_row;

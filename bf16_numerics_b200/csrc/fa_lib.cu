@@ -153,9 +153,10 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
     if (!set_smem(fa::fa_fwd_kernel<D>, L::SMEM_BYTES)) return FA_ERR_CUDA;
     attr = true;
   }
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
-    return cuda_fail("cuTensorMapEncodeTiled (q/k/v)");
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D) ||
+      !make_map(&mo, o, BH, N, D))
+    return cuda_fail("cuTensorMapEncodeTiled (q/k/v/o)");
   fa::FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -174,7 +175,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_qblk) * BH);
   LaunchTimer tm(FA_KERNEL_FWD, stream);
-  fa::fa_fwd_kernel<D><<<grid, 192, L::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  fa::fa_fwd_kernel<D><<<grid, 192, L::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
   tm.done();
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : cuda_fail("fa_fwd_kernel launch", e);
@@ -234,10 +235,12 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_blk) * BH);
     if (D == 64) {
-      CUtensorMap mdq;
+      CUtensorMap mdq, mdk, mdv;
       if (!make_map_dq(&mdq, dq_acc, BH, N)) return cuda_fail("cuTensorMapEncodeTiled (dQ accumulator)");
+      if (!make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
+        return cuda_fail("cuTensorMapEncodeTiled (dk/dv)");
       LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
-      fa::fa_bwd_main_pipe_kernel<<<grid, LP::THREADS, LP::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
+      fa::fa_bwd_main_pipe_kernel<<<grid, LP::THREADS, LP::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
       tm.done();
     } else {
       LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);

@@ -24,6 +24,12 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+// Profiling hook: a build that defines FA_TRACE_POINT(event) before including
+// this header can record per-CTA timelines; the library build compiles it out.
+#ifndef FA_TRACE_POINT
+#define FA_TRACE_POINT(event) ((void)0)
+#endif
+
 namespace fa {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -159,7 +165,10 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 // 32 lanes x 32 columns of 32-bit TMEM cells -> 32 registers per thread
 // (thread i of the warp gets lane base+i, register r holds column col+r).
 // The wait is inside the same asm statement so no use of the registers can be
-// scheduled before the data has arrived.
+// scheduled before the data has arrived.  TMEM accesses carry no "memory"
+// clobber (they touch no generic memory, so shared/global accesses may be
+// scheduled around them); being volatile, they stay ordered with respect to
+// the mbarrier waits and tcgen05 fences, which are volatile too.
 #define FA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -168,8 +177,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
       : FA_R8(0), FA_R8(8), FA_R8(16), FA_R8(24)
-      : "r"(taddr)
-      : "memory");
+      : "r"(taddr));
 }
 // Two 32-column loads, one wait.
 __device__ __forceinline__ void tmem_ld32x2(uint32_t taddr0, uint32_t taddr1, uint32_t (&r)[32], uint32_t (&s)[32]) {
@@ -183,8 +191,7 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t taddr0, uint32_t taddr1, ui
       "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
       : FA_R8(0), FA_R8(8), FA_R8(16), FA_R8(24), FA_S8(0), FA_S8(8), FA_S8(16), FA_S8(24)
-      : "r"(taddr0), "r"(taddr1)
-      : "memory");
+      : "r"(taddr0), "r"(taddr1));
 #undef FA_S8
 }
 #undef FA_R8
@@ -195,15 +202,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
       "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      FA_W8(0), FA_W8(8), FA_W8(16), FA_W8(24)
-      : "memory");
+      FA_W8(0), FA_W8(8), FA_W8(16), FA_W8(24));
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      FA_W8(0), FA_W8(8)
-      : "memory");
+      FA_W8(0), FA_W8(8));
 }
 #undef FA_W8
 __device__ __forceinline__ void tmem_st_wait() {
@@ -261,6 +266,8 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // wait until every committed bulk group has completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// wait until at most one committed bulk group is still in flight
+__device__ __forceinline__ void bulk_wait_all_but_one() { asm volatile("cp.async.bulk.wait_group 1;" ::: "memory"); }
 }  // namespace fa
 
 namespace fa {
@@ -305,12 +312,30 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       "tcgen05.wait::ld.sync.aligned;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
+      : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]));
+}
+}  // namespace fa
+
+namespace fa {
+// shared (128B-swizzled tile) -> global, tracked by the issuing thread's bulk group
+__device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(src), "r"(x), "r"(y), "r"(z)
                : "memory");
+}
+// One row (64 bf16 = 128 bytes, given as 32 packed bf16x2 words) of a
+// 128-row tile in the 128B-swizzled layout TMA uses: 16-byte chunk c of row r
+// lives at chunk c ^ (r & 7).  Conflict-free when consecutive threads write
+// consecutive rows.
+__device__ __forceinline__ void st_row_sw128(uint8_t* tile, int row, const uint32_t (&w)[32]) {
+  uint8_t* rp = tile + row * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4)) = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
 }
 }  // namespace fa
