@@ -26,7 +26,10 @@
 // TMEM columns: S^T[0] [0,128)  S^T[1] [128,256)  dP^T [256,384)
 //               dV [384,448)  dK [448,512)
 // Warps: 0-3 and 4-7 elementwise (key t = threadIdx % 128), 8-11 drain
-// (query t), 12 TMA producer, 13 MMA issuer / TMEM owner.
+// (query t), 12 TMA producer, 13 MMA issuer / TMEM owner, 14-15 idle.  The
+// block is launched with 128 registers per thread; the warpgroups then
+// re-balance them: elementwise 176, drain 96, TMA/MMA 56
+// (2*176 + 96 + 56 = 504 <= 4*128).
 #pragma once
 
 #include "fa_bwd.cuh"
@@ -60,7 +63,8 @@ struct BwdPipeLayout {
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512, DPT_COL = 256, DV_COL = 384, DK_COL = 448;
-  static constexpr int THREADS = 448;
+  static constexpr int THREADS = 512;
+  static constexpr uint32_t REGS_ELEM = 176, REGS_DRAIN = 96, REGS_CTRL = 56;
 };
 
 __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int x, int y, int z) {
@@ -71,7 +75,7 @@ __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src
       : "memory");
 }
 
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(512, 1)
 fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
@@ -85,7 +89,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   auto bar = [&](int i) { return base + L::BAR_OFF + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
-  float* vec = reinterpret_cast<float*>(smem + L::VEC_OFF);  // [s][0]: -a, [s][1]: 1/l, [s][2]: delta
+  // per-query vectors at VEC_OFF, [stage][0]: -a, [stage][1]: 1/l, [stage][2]: delta (fp32 x 128)
   const BoundedWait wait{abort_flag, 3u};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -127,6 +131,24 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) FA_TRACE_POINT(1);
 
+  // End of every role: all 16 warps meet on named barrier 15, then warp 13
+  // waits for its last MMAs and frees TMEM.  Each role's branch ends on its
+  // own (no common tail), so each keeps its own register budget.
+  auto teardown = [&]() {
+    tc_fence_before();
+    named_barrier_sync(15, L::THREADS);
+    if (threadIdx.x == 0) FA_TRACE_POINT(2);
+    if (warp == 13) {
+      tc_fence_after();
+      volatile int never = 0;
+      const BoundedWait drain{&never, 3u};
+      drain(bar(L::TEARDOWN), 0, 30);
+      tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+  };
+
+  if (warp >= 12) {
+    warpgroup_reg_dealloc<L::REGS_CTRL>();
   if (warp == 12) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -237,7 +259,12 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       tc_commit(bar(L::TEARDOWN));
     }
     __syncwarp();
-  } else if (warp >= 8) {
+  }  // warps 14-15: idle
+    teardown();
+    return;
+  }
+  if (warp >= 8) {
+    warpgroup_reg_dealloc<L::REGS_DRAIN>();
     // --------------------------------------------------------- drain warps
     const int t = threadIdx.x - 256;  // query within the block == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -268,9 +295,9 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           bb = 1.f;
         }
       }
-      vec[(s * 3 + 0) * 128 + t] = na;
-      vec[(s * 3 + 1) * 128 + t] = bb;
-      vec[(s * 3 + 2) * 128 + t] = dl;
+      sts32(base + L::VEC_OFF + ((s * 3 + 0) * 128 + t) * 4, na);
+      sts32(base + L::VEC_OFF + ((s * 3 + 1) * 128 + t) * 4, bb);
+      sts32(base + L::VEC_OFF + ((s * 3 + 2) * 128 + t) * 4, dl);
       mbar_arrive(bar(L::VEC_FULL + s));
     };
     if (n_it > 0) publish_vec(0, load_vec(0));
@@ -289,17 +316,19 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       if (t == 0) bulk_wait_read_all();  // the previous reduce has finished reading the staging tile
       named_barrier_sync(2, 128);
       // row t of each 32-column box, 16-byte chunk c stored at chunk c ^ (t & 7)
-      uint8_t* row0 = smem + L::DQS_OFF + t * 128;
-      uint8_t* row1 = row0 + TILE;
+      const uint32_t row0 = base + L::DQS_OFF + t * 128;
+      const uint32_t row1 = row0 + TILE;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const int pc = (c ^ (t & 7)) << 4;
-        *reinterpret_cast<float4*>(row0 + pc) =
-            make_float4(__uint_as_float(r0[4 * c]) * scale, __uint_as_float(r0[4 * c + 1]) * scale,
-                        __uint_as_float(r0[4 * c + 2]) * scale, __uint_as_float(r0[4 * c + 3]) * scale);
-        *reinterpret_cast<float4*>(row1 + pc) =
-            make_float4(__uint_as_float(r1[4 * c]) * scale, __uint_as_float(r1[4 * c + 1]) * scale,
-                        __uint_as_float(r1[4 * c + 2]) * scale, __uint_as_float(r1[4 * c + 3]) * scale);
+        const uint32_t pc = (c ^ (t & 7)) << 4;
+        sts128(row0 + pc, __float_as_uint(__uint_as_float(r0[4 * c]) * scale),
+               __float_as_uint(__uint_as_float(r0[4 * c + 1]) * scale),
+               __float_as_uint(__uint_as_float(r0[4 * c + 2]) * scale),
+               __float_as_uint(__uint_as_float(r0[4 * c + 3]) * scale));
+        sts128(row1 + pc, __float_as_uint(__uint_as_float(r1[4 * c]) * scale),
+               __float_as_uint(__uint_as_float(r1[4 * c + 1]) * scale),
+               __float_as_uint(__uint_as_float(r1[4 * c + 2]) * scale),
+               __float_as_uint(__uint_as_float(r1[4 * c + 3]) * scale));
       }
       fence_proxy_async_smem();
       named_barrier_sync(2, 128);
@@ -317,7 +346,11 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       }
     }
     if (t == 0) bulk_wait_all();
-  } else {
+    teardown();
+    return;
+  }
+  {
+    warpgroup_reg_alloc<L::REGS_ELEM>();
     // ----------------------------------------------- elementwise warps 0..7
     const int h = warp >> 2;          // query half
     const int t = threadIdx.x & 127;  // key within the block == TMEM lane
@@ -334,9 +367,9 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       if (!wait(bar(L::S_FULL + b), (i >> 1) & 1, 9)) { ok = false; break; }
       if (threadIdx.x == 0) FA_TRACE_POINT(20);
       tc_fence_after();
-      const float* va = vec + (b * 3 + 0) * 128 + 64 * h;
-      const float* vb = vec + (b * 3 + 1) * 128 + 64 * h;
-      const float* vd = vec + (b * 3 + 2) * 128 + 64 * h;
+      const uint32_t va = base + L::VEC_OFF + ((b * 3 + 0) * 128 + 64 * h) * 4;
+      const uint32_t vb = base + L::VEC_OFF + ((b * 3 + 1) * 128 + 64 * h) * 4;
+      const uint32_t vd = base + L::VEC_OFF + ((b * 3 + 2) * 128 + 64 * h) * 4;
       const bool diag = p.causal && (i0 + i == kblk);
       const int qoff = 64 * h;
       uint64_t p2[32];  // this row's 64 P values (fp32 pairs)
@@ -349,42 +382,42 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           p2[16 + e] = f2_pack(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
         }
       }
+      if (threadIdx.x == 0) FA_TRACE_POINT(25);
       // both warpgroups hold their S^T columns: P^T may now overwrite [0,64)
       named_barrier_sync(1, 256);
+      if (threadIdx.x == 0) FA_TRACE_POINT(26);
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const int pi = 8 * c + e, ql = 2 * pi;
-          const float4 na = *reinterpret_cast<const float4*>(va + ql);
-          const uint64_t y0 = f2_fma(p2[pi], C2, f2_pack(na.x, na.y));
-          const uint64_t y1 = f2_fma(p2[pi + 1], C2, f2_pack(na.z, na.w));
-          float a0, a1, a2, a3;
-          f2_unpack(y0, a0, a1);
-          f2_unpack(y1, a2, a3);
-          float p0 = ex2_approx(a0), p1 = ex2_approx(a1), p2v = ex2_approx(a2), p3 = ex2_approx(a3);
-          if (mode1) {
-            const float4 bb = *reinterpret_cast<const float4*>(vb + ql);
-            p0 *= bb.x;
-            p1 *= bb.y;
-            p2v *= bb.z;
-            p3 *= bb.w;
-          }
-          if (diag) {
-            const int qg = qoff + ql;
-            if (t > qg) p0 = 0.f;
-            if (t > qg + 1) p1 = 0.f;
-            if (t > qg + 2) p2v = 0.f;
-            if (t > qg + 3) p3 = 0.f;
-          }
-          p2[pi] = f2_pack(p0, p1);
-          p2[pi + 1] = f2_pack(p2v, p3);
-          pk[e] = pack_bf16x2(p0, p1);
-          pk[e + 1] = pack_bf16x2(p2v, p3);
+      for (int pi = 0; pi < 32; pi += 2) {
+        const int ql = 2 * pi;
+        const float4 na = lds128(va + ql * 4);
+        const uint64_t y0 = f2_fma(p2[pi], C2, f2_pack(na.x, na.y));
+        const uint64_t y1 = f2_fma(p2[pi + 1], C2, f2_pack(na.z, na.w));
+        float a0, a1, a2, a3;
+        f2_unpack(y0, a0, a1);
+        f2_unpack(y1, a2, a3);
+        float p0 = ex2_approx(a0), p1 = ex2_approx(a1), p2v = ex2_approx(a2), p3 = ex2_approx(a3);
+        if (mode1) {
+          const float4 bb = lds128(vb + ql * 4);
+          p0 *= bb.x;
+          p1 *= bb.y;
+          p2v *= bb.z;
+          p3 *= bb.w;
         }
-        tmem_st8(tmem + lane_base + 128u * b + 32u * h + 8u * c, pk);
+        if (diag) {
+          const int qg = qoff + ql;
+          if (t > qg) p0 = 0.f;
+          if (t > qg + 1) p1 = 0.f;
+          if (t > qg + 2) p2v = 0.f;
+          if (t > qg + 3) p3 = 0.f;
+        }
+        p2[pi] = f2_pack(p0, p1);
+        p2[pi + 1] = f2_pack(p2v, p3);
+        pk[pi] = pack_bf16x2(p0, p1);
+        pk[pi + 1] = pack_bf16x2(p2v, p3);
       }
+      tmem_st32(tmem + lane_base + 128u * b + 32u * h, pk);
+      if (threadIdx.x == 0) FA_TRACE_POINT(27);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::P_FULL + b));
@@ -394,36 +427,35 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       // the dQ product of the previous block has finished reading the dS tile
       if (i > 0 && !wait(bar(L::DQ_FULL + ((i - 1) & 1)), ((i - 1) >> 1) & 1, 11)) { ok = false; break; }
       tc_fence_after();
-      uint8_t* ds_row = smem + L::DS_OFF + h * TILE + t * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[16];
-        tmem_ld16(tmem + lane_base + L::DPT_COL + 64u * h + 16u * c, r);
-        uint32_t dk_[8];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const int pi = 8 * c + e, ql = 2 * pi;
-          const float4 dl = *reinterpret_cast<const float4*>(vd + ql);
-          const uint64_t ds0 = f2_mul(p2[pi], f2_sub(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])),
-                                                     f2_pack(dl.x, dl.y)));
-          const uint64_t ds1 = f2_mul(p2[pi + 1], f2_sub(f2_pack(__uint_as_float(r[2 * e + 2]), __uint_as_float(r[2 * e + 3])),
-                                                         f2_pack(dl.z, dl.w)));
-          float d0, d1, d2, d3;
-          f2_unpack(ds0, d0, d1);
-          f2_unpack(ds1, d2, d3);
-          dk_[e] = pack_bf16x2(d0, d1);
-          dk_[e + 1] = pack_bf16x2(d2, d3);
-        }
-        // dS^T into the dP^T columns this warpgroup has read: 64h + [0,32)
-        tmem_st8(tmem + lane_base + L::DPT_COL + 64u * h + 8u * c, dk_);
-        // dS^T row t, queries 64h + 16c + [0,16) = 16-byte chunks 2c, 2c+1 of the half tile
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int chunk = 2 * c + j;
-          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (t & 7)) << 4)) =
-              make_uint4(dk_[4 * j], dk_[4 * j + 1], dk_[4 * j + 2], dk_[4 * j + 3]);
-        }
+      const uint32_t ds_row = base + L::DS_OFF + h * TILE + t * 128;
+      uint32_t dpr[64];
+      {
+        uint32_t (&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]);
+        uint32_t (&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]);
+        tmem_ld32x2(tmem + lane_base + L::DPT_COL + 64u * h, tmem + lane_base + L::DPT_COL + 64u * h + 32u, d0, d1);
       }
+      uint32_t dk_[32];
+#pragma unroll
+      for (int pi = 0; pi < 32; pi += 2) {
+        const int ql = 2 * pi;
+        const float4 dl = lds128(vd + ql * 4);
+        const uint64_t ds0 = f2_mul(p2[pi], f2_sub(f2_pack(__uint_as_float(dpr[2 * pi]), __uint_as_float(dpr[2 * pi + 1])),
+                                                   f2_pack(dl.x, dl.y)));
+        const uint64_t ds1 = f2_mul(p2[pi + 1], f2_sub(f2_pack(__uint_as_float(dpr[2 * pi + 2]), __uint_as_float(dpr[2 * pi + 3])),
+                                                       f2_pack(dl.z, dl.w)));
+        float d0, d1, d2, d3;
+        f2_unpack(ds0, d0, d1);
+        f2_unpack(ds1, d2, d3);
+        dk_[pi] = pack_bf16x2(d0, d1);
+        dk_[pi + 1] = pack_bf16x2(d2, d3);
+      }
+      // dS^T into the dP^T columns this warpgroup has read: 64h + [0,32)
+      tmem_st32(tmem + lane_base + L::DPT_COL + 64u * h, dk_);
+      // dS^T row t, queries 64h + [0,64) = the eight 16-byte chunks of the half tile's row
+#pragma unroll
+      for (int chunk = 0; chunk < 8; ++chunk)
+        sts128(ds_row + ((chunk ^ (t & 7)) << 4), dk_[4 * chunk], dk_[4 * chunk + 1], dk_[4 * chunk + 2],
+               dk_[4 * chunk + 3]);
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
@@ -447,8 +479,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         w[c] = pack_bf16x2(__uint_as_float(r0[2 * c]) * f, __uint_as_float(r0[2 * c + 1]) * f);
         w[16 + c] = pack_bf16x2(__uint_as_float(r1[2 * c]) * f, __uint_as_float(r1[2 * c + 1]) * f);
       }
-      uint8_t* tile = smem + L::DS_OFF + h * TILE;
-      st_row_sw128(tile, t, w);
+      sts_row_sw128(base + L::DS_OFF + h * TILE, t, w);
       fence_proxy_async_smem();
       named_barrier_sync(3 + h, 128);
       if (t == 0) {
@@ -459,17 +490,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       }
     }
     (void)key;
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (threadIdx.x == 0) FA_TRACE_POINT(2);
-  if (warp == 13) {
-    tc_fence_after();
-    volatile int never = 0;
-    const BoundedWait drain{&never, 3u};
-    drain(bar(L::TEARDOWN), 0, 30);
-    tmem_dealloc(tmem, L::TMEM_COLS);
+    teardown();
   }
 }
 

@@ -91,6 +91,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int nkv = p.causal ? (qblk + 1) : n_kblk_all;
 
   if (threadIdx.x == 0) {
+    FA_TRACE_POINT(0);
     mbar_init(bar(L::Q_FULL), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(L::K_FULL + s), 1);
@@ -113,6 +114,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) FA_TRACE_POINT(1);
 
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
@@ -175,6 +177,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           if (!wait(bar(L::K_FULL + ((j + 1) & 1)), ((j + 1) >> 1) & 1, 3)) break;
           tc_fence_after();
           issue_s(j + 1);
+          FA_TRACE_POINT(10);
         }
         if (!wait(bar(L::P_FULL), j & 1, 5)) break;
         if (!wait(bar(L::V_FULL + s), (j >> 1) & 1, 6)) break;
@@ -186,6 +189,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         tc_commit(bar(L::O_READY));
         tc_commit(bar(L::KV_EMPTY + s));
+        FA_TRACE_POINT(11);
       }
       tc_commit(bar(L::TEARDOWN));
     }
@@ -208,6 +212,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       if (!wait(bar(L::S_FULL), j & 1, 7)) { ok = false; break; }
+      if (t == 0) FA_TRACE_POINT(20);
       tc_fence_after();
       float x[128];
       {
@@ -222,6 +227,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       tc_fence_before();
       mbar_arrive(bar(L::S_FREE));
+      if (t == 0) FA_TRACE_POINT(21);
       // mask (diagonal tile / ragged tail) and tile max, eight partial maxima
       const int kv0 = j * L::BN;
       const bool diag = p.causal && (j == qblk);
@@ -265,8 +271,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       float m_new = rm_s;
       if (p.mode == 1 && rs > 1) m_new = (rm_s > 0.f) ? beta * rm_s : ((rm_s < 0.f) ? 0.f : beta - 1.f);
       // P and O are free once the previous P V product has completed
+      if (t == 0) FA_TRACE_POINT(22);
       if (j > 0) {
         if (!wait(bar(L::O_READY), (j - 1) & 1, 8)) { ok = false; break; }
+        if (t == 0) FA_TRACE_POINT(23);
         tc_fence_after();
         const bool changed = (m_new != m_run);
         float alpha = 1.f;
@@ -315,6 +323,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::P_FULL));
+      if (t == 0) FA_TRACE_POINT(24);
     }
     // ------------------------------------------------------------- epilogue
     if (ok && nkv > 0 && wait(bar(L::O_READY), (nkv - 1) & 1, 9)) {
@@ -333,7 +342,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           w[c] = pack_bf16x2(__uint_as_float(r0[2 * c]) * inv_l, __uint_as_float(r0[2 * c + 1]) * inv_l);
           w[16 + c] = pack_bf16x2(__uint_as_float(r1[2 * c]) * inv_l, __uint_as_float(r1[2 * c + 1]) * inv_l);
         }
-        st_row_sw128(smem + L::K_OFF + h * L::HALF, t, w);
+        sts_row_sw128(base + L::K_OFF + h * L::HALF, t, w);
       }
       fence_proxy_async_smem();
       named_barrier_sync(1, 128);
@@ -357,6 +366,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   // ----------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) FA_TRACE_POINT(2);
   if (warp == 5) {
     tc_fence_after();
     volatile int never = 0;

@@ -339,3 +339,41 @@ __device__ __forceinline__ void st_row_sw128(uint8_t* tile, int row, const uint3
     *reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4)) = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
 }
 }  // namespace fa
+
+namespace fa {
+// Register re-balancing between warpgroups (all four warps of a warpgroup
+// execute the same instruction).  The block is launched with a fixed per-thread
+// count; the warpgroups' new counts must sum to no more than four times it.
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+}  // namespace fa
+
+namespace fa {
+// Explicit shared-memory accesses by 32-bit shared address (ld/st.shared), so
+// no access through a generic pointer can fall back to the generic path.
+// (not volatile: free to be scheduled among arithmetic and TMEM accesses; the
+// "memory" clobber keeps it after the mbarrier waits that publish the data)
+__device__ __forceinline__ float4 lds128(uint32_t addr) {
+  float4 v;
+  asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ void sts32(uint32_t addr, float a) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(a) : "memory");
+}
+// st_row_sw128 with an explicit shared address
+__device__ __forceinline__ void sts_row_sw128(uint32_t tile, int row, const uint32_t (&w)[32]) {
+  const uint32_t rp = tile + row * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) sts128(rp + ((c ^ (row & 7)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+}
+}  // namespace fa
