@@ -50,6 +50,8 @@ fa_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __
   const long long warp_global = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const int sub = lane / LPR, li = lane % LPR;
+  grid_launch_dependents();
+  grid_dependency_wait();  // O comes from the forward grid
   for (long long r0 = warp_global * RPW; r0 < rows; r0 += n_warps * RPW) {
     const long long r = r0 + sub;
     float acc = 0.f;
@@ -79,6 +81,8 @@ fa_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __
 __global__ void __launch_bounds__(256)
 fa_bwd_dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq, long long n8) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  grid_launch_dependents();
+  grid_dependency_wait();  // the accumulator is complete once the main grid is
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
     const float4 a = __ldg(reinterpret_cast<const float4*>(dq_acc) + 2 * i);
     const float4 b = __ldg(reinterpret_cast<const float4*>(dq_acc) + 2 * i + 1);
@@ -172,6 +176,8 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
+  grid_launch_dependents();
+  grid_dependency_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -125,6 +125,8 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
+  grid_launch_dependents();
+  grid_dependency_wait();  // delta and the cleared dQ accumulator come from the previous grid
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

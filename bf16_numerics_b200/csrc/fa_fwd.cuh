@@ -110,6 +110,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
+  grid_launch_dependents();
+  // inputs (and the outputs' previous contents) belong to the previous grid in
+  // the stream until it has completed: everything above overlaps its tail
+  grid_dependency_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -235,31 +239,36 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const int lim_len = p.N - 1 - kv0;
       const int lim = lim_causal < lim_len ? lim_causal : lim_len;
       const bool masked = (lim < L::BN - 1);
+      // tile max: three-input max, eight partial maxima
       float pm[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
       if (masked) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float v = (c <= lim) ? x[c] * cmp_scale : -INFINITY;
-          x[c] = v;
-          pm[c & 7] = fmaxf(pm[c & 7], v);
-        }
-      } else {
+        for (int c = 0; c < 128; ++c) x[c] = (c <= lim) ? x[c] * cmp_scale : -INFINITY;
+      } else if (!kRawCompare) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          if (!kRawCompare) x[c] *= cmp_scale;
-          pm[c & 7] = fmaxf(pm[c & 7], x[c]);
-        }
+        for (int c = 0; c < 128; ++c) x[c] *= cmp_scale;
       }
-      const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      // tie count: only rows whose tile max reaches the running max need it
-      if (__any_sync(0xffffffffu, tmax >= rm_x)) {
-        int cnt[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int c = 0; c < 128; ++c) cnt[c & 3] += (x[c] == tmax) ? 1 : 0;
-        const int tc = (cnt[0] + cnt[1]) + (cnt[2] + cnt[3]);
+      for (int c = 0; c < 128; c += 16) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) pm[u] = fmax3(pm[u], x[c + 2 * u], x[c + 2 * u + 1]);
+      }
+      const float tmax = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+      // tie count: only rows whose tile max reaches the running max need it;
+      // set.eq gives 1.0/0.0, summed exactly in fp32 pairs (counts <= 128)
+      if (__any_sync(0xffffffffu, tmax >= rm_x)) {
+        uint64_t cnt2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int c = 0; c < 128; c += 2)
+          cnt2[(c >> 1) & 3] = f2_add(cnt2[(c >> 1) & 3], f2_pack(feq(x[c], tmax), feq(x[c + 1], tmax)));
+        float c0, c1, c2, c3, c4, c5, c6, c7;
+        f2_unpack(cnt2[0], c0, c1);
+        f2_unpack(cnt2[1], c2, c3);
+        f2_unpack(cnt2[2], c4, c5);
+        f2_unpack(cnt2[3], c6, c7);
+        const int tc = static_cast<int>(((c0 + c1) + (c2 + c3)) + ((c4 + c5) + (c6 + c7)));
         if (tmax > rm_x) {
           rm_x = tmax;
           rs = tc;

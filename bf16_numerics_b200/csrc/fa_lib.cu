@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "fa_b200.h"
@@ -125,6 +126,26 @@ struct LaunchTimer {
   }
 };
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream is finishing; every kernel of this
+// library executes griddepcontrol.wait before touching data the previous
+// grid may still be producing.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <typename K>
 bool set_smem(K kernel, int bytes) {
   const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -175,9 +196,9 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_qblk) * BH);
   LaunchTimer tm(FA_KERNEL_FWD, stream);
-  fa::fa_fwd_kernel<D><<<grid, 192, L::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+  cudaError_t e = launch_pdl(fa::fa_fwd_kernel<D>, dim3(grid), dim3(192), L::SMEM_BYTES, stream, mq, mk, mv, mo, p);
   tm.done();
-  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : cuda_fail("fa_fwd_kernel launch", e);
 }
 
@@ -213,10 +234,11 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   {
     constexpr int rows_per_block = 8 * (32 / (D / 8));
     LaunchTimer tm(FA_KERNEL_BWD_DELTA, stream);
-    fa::fa_bwd_delta_kernel<D><<<grid_for(rows, rows_per_block), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows);
+    cudaError_t e = launch_pdl(fa::fa_bwd_delta_kernel<D>, dim3(grid_for(rows, rows_per_block)), dim3(256), 0,
+                               stream, static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO),
+                               delta, dq_acc, rows);
     tm.done();
-    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("fa_bwd_delta_kernel launch", e);
   }
   {
@@ -240,23 +262,29 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       if (!make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
         return cuda_fail("cuTensorMapEncodeTiled (dk/dv)");
       LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
-      fa::fa_bwd_main_pipe_kernel<<<grid, LP::THREADS, LP::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
+      cudaError_t e = launch_pdl(fa::fa_bwd_main_pipe_kernel, dim3(grid), dim3(LP::THREADS), LP::SMEM_BYTES, stream,
+                                 mq, mk, mv, mdo, mdq, mdk, mdv, p);
       tm.done();
+      if (e == cudaSuccess) e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
     } else {
       LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
-      fa::fa_bwd_main_kernel<D><<<grid, 320, L::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
+      cudaError_t e = launch_pdl(fa::fa_bwd_main_kernel<D>, dim3(grid), dim3(320), L::SMEM_BYTES, stream, mq, mk, mv,
+                                 mdo, p);
       tm.done();
+      if (e == cudaSuccess) e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
     }
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = cudaSuccess;
     if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
   }
   {
     const long long n8 = rows * D / 8;
     LaunchTimer tm(FA_KERNEL_BWD_DQ, stream);
-    fa::fa_bwd_dq_convert_kernel<<<grid_for(n8, 256), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
-                                                                         n8);
+    cudaError_t e = launch_pdl(fa::fa_bwd_dq_convert_kernel, dim3(grid_for(n8, 256)), dim3(256), 0, stream,
+                               static_cast<const float*>(dq_acc), static_cast<__nv_bfloat16*>(dq), n8);
     tm.done();
-    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("fa_bwd_dq_convert_kernel launch", e);
   }
   return FA_OK;

@@ -377,3 +377,26 @@ __device__ __forceinline__ void sts_row_sw128(uint32_t tile, int row, const uint
   for (int c = 0; c < 8; ++c) sts128(rp + ((c ^ (row & 7)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
 }
 }  // namespace fa
+
+namespace fa {
+// three-input maximum (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// 1.0f if a == b, else 0.0f
+__device__ __forceinline__ float feq(float a, float b) {
+  float r;
+  asm("set.eq.f32.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+}  // namespace fa
+
+namespace fa {
+// Programmatic dependent launch: wait until the grid this one depends on has
+// completed and its memory is visible (no-op when launched without the
+// attribute), and allow the next grid in the stream to be scheduled.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+}  // namespace fa
