@@ -1,13 +1,17 @@
-// Pipelined backward main kernel for head dimension 64.
+// Persistent, pipelined backward main kernel for head dimension 64.
 //
-// Same mathematics as fa_bwd_main_kernel (see fa_bwd.cuh): one CTA per
-// (batch, head, 128-key block), looping over the query blocks that see the
-// keys, in the transposed orientation (lane = key).  What changes is the
-// schedule, so that the tensor core and the elementwise work overlap:
+// Same mathematics as fa_bwd_main_kernel (see fa_bwd.cuh): the work is split
+// into items = (batch*head, 128-key block); an item loops over the query blocks
+// that see its keys, in the transposed orientation (lane = key).  One CTA per
+// SM walks a list of items (snake order over the CTAs, items sorted by
+// decreasing work), so TMEM allocation and barrier set-up happen once per CTA
+// and the K/V loads and first products of an item overlap the previous item's
+// dK/dV epilogue.
 //
+// Within an item, the schedule overlaps tensor core and elementwise work:
 //   * S^T is double-buffered in TMEM: the MMA warp issues S^T of query block
-//     i+2 while the elementwise warps work on block i, and dP^T of block i+1
-//     as soon as block i's dS has been consumed.
+//     g+2 while the elementwise warps work on block g, and dP^T of block g+1
+//     as soon as block g's dS has been consumed.
 //   * Eight elementwise warps (two warpgroups) split the 128 query columns of
 //     a key row: warpgroup h takes columns [64h, 64h+64).  Both copy their S^T
 //     columns to registers and meet at a named barrier; then warpgroup h
@@ -15,21 +19,26 @@
 //     [0,64) and [64,128) is free for dQ.  dS^T goes into the first half of
 //     the dP^T columns each warpgroup has just read (64h + [0,32)), which
 //     needs no barrier.
-//   * dQ_i = dS K is one N = 64 product into S^T cols [64,128) of the same
-//     buffer, which no later product of the iteration touches.
+//   * dQ_g = dS K is one N = 64 product into S^T cols [64,128) of the same
+//     buffer, which no later product of the block touches.
 //   * Four drain warps move the dQ partial from TMEM into a 128B-swizzled
 //     fp32 tile in shared memory and add it to the fp32 accumulator in global
 //     memory with one TMA tensor reduce-add per 32-column half (rows past N
 //     are clipped by the tensor map).  They also prepare the per-query
 //     vectors (lse or m, 1/l, delta) two blocks ahead.
 //
+// Barrier phases count a global query-block index g that runs across the
+// CTA's items; every phase of every barrier is waited for in order and no
+// producer can get two phases ahead of a consumer's wait (the MMA warp waits
+// for the drain's release of block g right after issuing dQ_g, before dQ_g+1).
+//
 // TMEM columns: S^T[0] [0,128)  S^T[1] [128,256)  dP^T [256,384)
 //               dV [384,448)  dK [448,512)
 // Warps: 0-3 and 4-7 elementwise (key t = threadIdx % 128), 8-11 drain
 // (query t), 12 TMA producer, 13 MMA issuer / TMEM owner, 14-15 idle.  The
 // block is launched with 128 registers per thread; the warpgroups then
-// re-balance them: elementwise 176, drain 96, TMA/MMA 56
-// (2*176 + 96 + 56 = 504 <= 4*128).
+// re-balance them: elementwise 168, drain 88, TMA/MMA 88
+// (2*168 + 88 + 88 = 512 = 4*128).
 #pragma once
 
 #include "fa_bwd.cuh"
@@ -46,17 +55,19 @@ struct BwdPipeLayout {
   static constexpr int BAR_OFF = VEC_OFF + 2 * 3 * 128 * 4;
   enum {
     KV_FULL = 0,
-    Q_FULL = 1,
+    KV_EMPTY,
+    Q_FULL,
     Q_EMPTY = Q_FULL + NST,
-    S_FULL = Q_EMPTY + NST,  // [2]
-    P_FULL = S_FULL + 2,     // [2]
+    S_FULL = Q_EMPTY + NST,    // [2]
+    P_FULL = S_FULL + 2,       // [2]
     DP_FULL = P_FULL + 2,
     DS_FULL,
-    DQ_FULL,                 // [2]
+    DQ_FULL,                   // [2]
     DQ_FREE = DQ_FULL + 2,
-    VEC_FULL,                // [2]
+    VEC_FULL,                  // [2]
     VEC_EMPTY = VEC_FULL + 2,  // [2]
     ACC_DONE = VEC_EMPTY + 2,
+    ACC_FREE,
     TEARDOWN,
     NBAR
   };
@@ -64,7 +75,7 @@ struct BwdPipeLayout {
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512, DPT_COL = 256, DV_COL = 384, DK_COL = 448;
   static constexpr int THREADS = 512;
-  static constexpr uint32_t REGS_ELEM = 176, REGS_DRAIN = 96, REGS_CTRL = 56;
+  static constexpr uint32_t REGS_ELEM = 168, REGS_DRAIN = 88, REGS_CTRL = 88;
 };
 
 __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int x, int y, int z) {
@@ -74,6 +85,48 @@ __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src
       "r"(src), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+
+// Items of one CTA: the r-th is item number r*G + c (r even) or
+// r*G + G-1-c (r odd) of the list sorted by decreasing work (key block 0
+// first when causal), G = gridDim.x.  Item number w is key block w / BH of
+// batch*head w % BH.  The cursor walks (item, query block) pairs in order.
+struct BwdCursor {
+  int c, G, W, BH, n_blk, causal;
+  int r, kblk, bh, n, i0, i;
+  bool valid;
+  __device__ __forceinline__ void load() {
+    const int w = r * G + ((r & 1) ? (G - 1 - c) : c);
+    valid = w < W;
+    if (valid) {
+      kblk = w / BH;
+      bh = w - kblk * BH;
+      n = causal ? (n_blk - kblk) : n_blk;
+      i0 = causal ? kblk : 0;
+      i = 0;
+    }
+  }
+  __device__ __forceinline__ void start(const BwdParams& p) {
+    c = blockIdx.x;
+    G = gridDim.x;
+    BH = p.BH;
+    n_blk = p.n_blk;
+    W = p.n_blk * p.BH;
+    causal = p.causal;
+    r = 0;
+    load();
+  }
+  __device__ __forceinline__ void next_block() {
+    if (++i >= n) {
+      ++r;
+      load();
+    }
+  }
+  __device__ __forceinline__ void next_item() {
+    ++r;
+    load();
+  }
+  __device__ __forceinline__ int qblk() const { return i0 + i; }
+};
 
 __global__ void __launch_bounds__(512, 1)
 fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -91,17 +144,12 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   // per-query vectors at VEC_OFF, [stage][0]: -a, [stage][1]: 1/l, [stage][2]: delta (fp32 x 128)
   const BoundedWait wait{abort_flag, 3u};
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = p.BH;
-  const int kblk = blockIdx.x / BH;
-  const int bh = blockIdx.x - kblk * BH;
-  const int i0 = p.causal ? kblk : 0;
-  const int n_it = p.n_blk - i0;
 
   if (threadIdx.x == 0) {
     FA_TRACE_POINT(0);
     mbar_init(bar(L::KV_FULL), 1);
+    mbar_init(bar(L::KV_EMPTY), 1);
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar(L::Q_FULL + s), 1);
       mbar_init(bar(L::Q_EMPTY + s), 1);
@@ -117,6 +165,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     mbar_init(bar(L::DS_FULL), 256);
     mbar_init(bar(L::DQ_FREE), 128);
     mbar_init(bar(L::ACC_DONE), 1);
+    mbar_init(bar(L::ACC_FREE), 256);
     mbar_init(bar(L::TEARDOWN), 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -151,141 +200,166 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
 
   if (warp >= 12) {
     warpgroup_reg_dealloc<L::REGS_CTRL>();
-  if (warp == 12) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (warp == 12 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_expect_tx(bar(L::KV_FULL), 2 * TILE);
-      tma_load_3d(base + L::K_OFF, &tm_k, bar(L::KV_FULL), 0, kblk * L::B, bh);
-      tma_load_3d(base + L::V_OFF, &tm_v, bar(L::KV_FULL), 0, kblk * L::B, bh);
+      BwdCursor cur;
+      cur.start(p);
+      int g = 0, last_r = -1;
       int issued[NST];
       for (int s = 0; s < NST; ++s) issued[s] = -1;
-      for (int i = 0; i < n_it; ++i) {
-        const int s = i % NST, use = i / NST;
-        if (use > 0 && !wait(bar(L::Q_EMPTY + s), (use - 1) & 1, 1)) break;
-        const int row0 = (i0 + i) * L::B;
+      auto load_q = [&](int i, int gq) {
+        const int s = gq % NST, use = gq / NST;
+        if (use > 0 && !wait(bar(L::Q_EMPTY + s), (use - 1) & 1, 1)) return false;
+        const int row0 = (cur.i0 + i) * L::B;
         mbar_expect_tx(bar(L::Q_FULL + s), 2 * TILE);
-        tma_load_3d(base + L::Q_OFF + s * TILE, &tm_q, bar(L::Q_FULL + s), 0, row0, bh);
-        tma_load_3d(base + L::DO_OFF + s * TILE, &tm_do, bar(L::Q_FULL + s), 0, row0, bh);
-        issued[s] = i;
+        tma_load_3d(base + L::Q_OFF + s * TILE, &tm_q, bar(L::Q_FULL + s), 0, row0, cur.bh);
+        tma_load_3d(base + L::DO_OFF + s * TILE, &tm_do, bar(L::Q_FULL + s), 0, row0, cur.bh);
+        issued[s] = gq;
+        return true;
+      };
+      bool ok = true;
+      for (; ok && cur.valid; cur.next_item()) {
+        // the item's first query blocks go ahead of its K/V, which must wait
+        // for the previous item's products to release the K/V buffers
+        const int first = cur.n < 2 ? cur.n : 2;
+        for (int i = 0; ok && i < first; ++i) ok = load_q(i, g + i);
+        if (!ok) break;
+        if (cur.r > 0 && !wait(bar(L::KV_EMPTY), (cur.r - 1) & 1, 1)) break;
+        mbar_expect_tx(bar(L::KV_FULL), 2 * TILE);
+        tma_load_3d(base + L::K_OFF, &tm_k, bar(L::KV_FULL), 0, cur.kblk * L::B, cur.bh);
+        tma_load_3d(base + L::V_OFF, &tm_v, bar(L::KV_FULL), 0, cur.kblk * L::B, cur.bh);
+        last_r = cur.r;
+        for (int i = first; ok && i < cur.n; ++i) ok = load_q(i, g + i);
+        g += cur.n;
       }
       volatile int never = 0;
       const BoundedWait drain{&never, 3u};
-      drain(bar(L::KV_FULL), 0, 20);
+      if (last_r >= 0) drain(bar(L::KV_FULL), last_r & 1, 20);
       for (int s = 0; s < NST; ++s)
         if (issued[s] >= 0) drain(bar(L::Q_FULL + s), (issued[s] / NST) & 1, 21);
-    }
-    __syncwarp();
-  } else if (warp == 13) {
-    // -------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    } else if (warp == 13 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t IDESC_SQ = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 64, false, true);    // dV, dK
       constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, 64, true, true);     // dQ
-      auto q_tile = [&](int i) { return base + L::Q_OFF + (i % NST) * TILE; };
-      auto do_tile = [&](int i) { return base + L::DO_OFF + (i % NST) * TILE; };
-      auto issue_s = [&](int i) {
-        const uint32_t d_tmem = tmem + 128u * (i & 1);
+      auto q_tile = [&](int g) { return base + L::Q_OFF + (g % NST) * TILE; };
+      auto do_tile = [&](int g) { return base + L::DO_OFF + (g % NST) * TILE; };
+      auto issue_s = [&](int g) {
+        const uint32_t d_tmem = tmem + 128u * (g & 1);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_ss(d_tmem, sdesc_sw128(base + L::K_OFF + ks * 32, 16, 1024), sdesc_sw128(q_tile(i) + ks * 32, 16, 1024),
+          mma_ss(d_tmem, sdesc_sw128(base + L::K_OFF + ks * 32, 16, 1024), sdesc_sw128(q_tile(g) + ks * 32, 16, 1024),
                  IDESC_SQ, ks > 0 ? 1u : 0u);
-        tc_commit(bar(L::S_FULL + (i & 1)));
+        tc_commit(bar(L::S_FULL + (g & 1)));
       };
-      auto issue_dp = [&](int i) {
+      auto issue_dp = [&](int g) {
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_ss(tmem + L::DPT_COL, sdesc_sw128(base + L::V_OFF + ks * 32, 16, 1024),
-                 sdesc_sw128(do_tile(i) + ks * 32, 16, 1024), IDESC_SQ, ks > 0 ? 1u : 0u);
+                 sdesc_sw128(do_tile(g) + ks * 32, 16, 1024), IDESC_SQ, ks > 0 ? 1u : 0u);
         tc_commit(bar(L::DP_FULL));
       };
-      bool ok = wait(bar(L::KV_FULL), 0, 2);
-      if (ok && n_it > 0) {
-        ok = wait(bar(L::Q_FULL + 0), 0, 3);
-        if (ok) {
-          tc_fence_after();
-          issue_s(0);
-          issue_dp(0);
-        }
-      }
-      if (ok && n_it > 1) {
-        ok = wait(bar(L::Q_FULL + 1), 0, 3);
-        if (ok) {
-          tc_fence_after();
-          issue_s(1);
-        }
-      }
-      for (int i = 0; ok && i < n_it; ++i) {
-        const int b = i & 1;
-        if (!wait(bar(L::P_FULL + b), (i >> 1) & 1, 4)) break;
-        FA_TRACE_POINT(10);
+      BwdCursor cur;
+      cur.start(p);
+      int g0 = 0;
+      bool ok = true;
+      for (; ok && cur.valid; cur.next_item()) {
+        const int n = cur.n;
+        if (!wait(bar(L::KV_FULL), cur.r & 1, 2)) break;
+        // S^T of this item's first two blocks (their TMEM buffers were released
+        // by the drain waits of the previous item), dP^T of the first
+        if (!wait(bar(L::Q_FULL + (g0 % NST)), (g0 / NST) & 1, 3)) break;
         tc_fence_after();
-        // dV += P^T dO_i   (K-dim = queries; P^T at S^T cols [0,64))
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t a = tmem + 128u * b + 8u * ks;
-          mma_ts(tmem + L::DV_COL, a, sdesc_sw128(do_tile(i) + ks * 2048, 16384, 1024), IDESC_KV,
-                 (i > 0 || ks > 0) ? 1u : 0u);
+        issue_s(g0);
+        issue_dp(g0);
+        if (n > 1) {
+          if (!wait(bar(L::Q_FULL + ((g0 + 1) % NST)), ((g0 + 1) / NST) & 1, 3)) break;
+          tc_fence_after();
+          issue_s(g0 + 1);
         }
-        if (!wait(bar(L::DS_FULL), i & 1, 5)) break;
-        FA_TRACE_POINT(11);
-        tc_fence_after();
-        // dK += dS^T Q_i
+        for (int i = 0; i < n; ++i) {
+          const int g = g0 + i, b = g & 1;
+          if (!wait(bar(L::P_FULL + b), (g >> 1) & 1, 4)) { ok = false; break; }
+          FA_TRACE_POINT(10);
+          // the first dV product of an item overwrites the accumulators: the
+          // previous item's epilogue must have copied them out
+          if (i == 0 && cur.r > 0 && !wait(bar(L::ACC_FREE), (cur.r - 1) & 1, 8)) { ok = false; break; }
+          tc_fence_after();
+          // dV += P^T dO_g   (K-dim = queries; P^T at S^T cols [0,64))
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t a = tmem + L::DPT_COL + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4));
-          mma_ts(tmem + L::DK_COL, a, sdesc_sw128(q_tile(i) + ks * 2048, 16384, 1024), IDESC_KV,
-                 (i > 0 || ks > 0) ? 1u : 0u);
-        }
-        // dQ_i = dS K into S^T cols [64,128) of the same buffer
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ts(tmem + L::DV_COL, tmem + 128u * b + 8u * ks, sdesc_sw128(do_tile(g) + ks * 2048, 16384, 1024),
+                   IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
+          if (!wait(bar(L::DS_FULL), g & 1, 5)) { ok = false; break; }
+          FA_TRACE_POINT(11);
+          tc_fence_after();
+          // dK += dS^T Q_g
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ss(tmem + 128u * b + 64u, sdesc_sw128(base + L::DS_OFF + ks * 2048, 16384, 1024),
-                 sdesc_sw128(base + L::K_OFF + ks * 2048, 16384, 1024), IDESC_DQ, ks > 0 ? 1u : 0u);
-        tc_commit(bar(L::DQ_FULL + b));
-        tc_commit(bar(L::Q_EMPTY + (i % NST)));
-        if (i + 1 < n_it) issue_dp(i + 1);
-        FA_TRACE_POINT(12);
-        if (i + 2 < n_it) {
-          if (!wait(bar(L::DQ_FREE), i & 1, 6)) break;
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t a = tmem + L::DPT_COL + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4));
+            mma_ts(tmem + L::DK_COL, a, sdesc_sw128(q_tile(g) + ks * 2048, 16384, 1024), IDESC_KV,
+                   (i > 0 || ks > 0) ? 1u : 0u);
+          }
+          // dQ_g = dS K into S^T cols [64,128) of the same buffer
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + 128u * b + 64u, sdesc_sw128(base + L::DS_OFF + ks * 2048, 16384, 1024),
+                   sdesc_sw128(base + L::K_OFF + ks * 2048, 16384, 1024), IDESC_DQ, ks > 0 ? 1u : 0u);
+          tc_commit(bar(L::DQ_FULL + b));
+          tc_commit(bar(L::Q_EMPTY + (g % NST)));
+          if (i + 1 < n) {
+            issue_dp(g + 1);
+          } else {
+            tc_commit(bar(L::ACC_DONE));  // dV, dK of this item complete
+            tc_commit(bar(L::KV_EMPTY));  // K, V of this item no longer read
+          }
+          FA_TRACE_POINT(12);
+          // dQ_g drained from TMEM: its S^T buffer may take block g+2
+          if (!wait(bar(L::DQ_FREE), g & 1, 6)) { ok = false; break; }
           FA_TRACE_POINT(13);
-          if (!wait(bar(L::Q_FULL + ((i + 2) % NST)), ((i + 2) / NST) & 1, 7)) break;
-          tc_fence_after();
-          issue_s(i + 2);
+          if (i + 2 < n) {
+            if (!wait(bar(L::Q_FULL + ((g + 2) % NST)), ((g + 2) / NST) & 1, 7)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(g + 2);
+          }
         }
+        g0 += n;
       }
-      tc_commit(bar(L::ACC_DONE));
       tc_commit(bar(L::TEARDOWN));
     }
     __syncwarp();
-  }  // warps 14-15: idle
     teardown();
     return;
   }
+
   if (warp >= 8) {
     warpgroup_reg_dealloc<L::REGS_DRAIN>();
-    // --------------------------------------------------------- drain warps
+    // ----------------------------------------------------------- drain warps
     const int t = threadIdx.x - 256;  // query within the block == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float scale = p.scale;
-    const size_t vrow0 = static_cast<size_t>(bh) * p.N;
-    // per-query vectors of block i: global loads first (prefetch), smem later
-    struct Vec3 { float lse, m, dl; };
-    auto load_vec = [&](int i) {
+    struct Vec3 {
+      float lse, m, dl;
+    };
+    auto load_vec = [&](const BwdCursor& c) {
       Vec3 v{0.f, 0.f, 0.f};
-      const int q = (i0 + i) * L::B + t;
-      if (i < n_it && q < p.N) {
-        v.lse = __ldg(p.lse + vrow0 + q);
-        v.dl = __ldg(p.delta + vrow0 + q);
-        v.m = (p.mode == 1) ? __ldg(p.row_m + vrow0 + q) : 0.f;
+      if (c.valid) {
+        const int q = c.qblk() * L::B + t;
+        if (q < p.N) {
+          const size_t vi = static_cast<size_t>(c.bh) * p.N + q;
+          v.lse = __ldg(p.lse + vi);
+          v.dl = __ldg(p.delta + vi);
+          v.m = (p.mode == 1) ? __ldg(p.row_m + vi) : 0.f;
+        }
       }
       return v;
     };
-    auto publish_vec = [&](int i, const Vec3& v) {
-      const int s = i & 1, q = (i0 + i) * L::B + t;
+    auto publish_vec = [&](int g, const BwdCursor& c, const Vec3& v) {
+      const int s = g & 1, q = c.qblk() * L::B + t;
       float na = -INFINITY, bb = 0.f, dl = 0.f;
       if (q < p.N) {
         dl = v.dl;
@@ -302,13 +376,18 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       sts32(base + L::VEC_OFF + ((s * 3 + 2) * 128 + t) * 4, dl);
       mbar_arrive(bar(L::VEC_FULL + s));
     };
-    if (n_it > 0) publish_vec(0, load_vec(0));
-    if (n_it > 1) publish_vec(1, load_vec(1));
-    Vec3 next = load_vec(2);
+    // pub walks two blocks ahead of cur, nxt holds the loads for pub
+    BwdCursor cur, pub;
+    cur.start(p);
+    pub.start(p);
+    int g_pub = 0;
+    for (int k = 0; k < 2 && pub.valid; ++k, ++g_pub, pub.next_block()) publish_vec(g_pub, pub, load_vec(pub));
+    Vec3 nxt = load_vec(pub);
     if (t == 0) tma_prefetch_desc(&tm_dq);
-    for (int i = 0; i < n_it; ++i) {
-      const int b = i & 1;
-      if (!wait(bar(L::DQ_FULL + b), (i >> 1) & 1, 13)) break;
+    bool ok = true;
+    for (int g = 0; ok && cur.valid; ++g, cur.next_block()) {
+      const int b = g & 1;
+      if (!wait(bar(L::DQ_FULL + b), (g >> 1) & 1, 13)) break;
       if (t == 0) FA_TRACE_POINT(30);
       tc_fence_after();
       uint32_t r0[32], r1[32];
@@ -335,146 +414,159 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       fence_proxy_async_smem();
       named_barrier_sync(2, 128);
       if (t == 0) {
-        const int q0 = (i0 + i) * L::B;
-        tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF, 0, q0, bh);
-        tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF + TILE, 32, q0, bh);
+        const int q0 = cur.qblk() * L::B;
+        tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF, 0, q0, cur.bh);
+        tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF + TILE, 32, q0, cur.bh);
         bulk_commit();
         FA_TRACE_POINT(31);
       }
-      if (i + 2 < n_it) {
-        if (!wait(bar(L::VEC_EMPTY + b), (i >> 1) & 1, 14)) break;
-        publish_vec(i + 2, next);
-        next = load_vec(i + 3);
+      if (pub.valid) {
+        // block g+2 reuses the vector stage of block g
+        if (!wait(bar(L::VEC_EMPTY + b), (g >> 1) & 1, 14)) { ok = false; break; }
+        publish_vec(g_pub, pub, nxt);
+        ++g_pub;
+        pub.next_block();
+        nxt = load_vec(pub);
       }
     }
     if (t == 0) bulk_wait_all();
     teardown();
     return;
   }
+
   {
     warpgroup_reg_alloc<L::REGS_ELEM>();
-    // ----------------------------------------------- elementwise warps 0..7
+    // ------------------------------------------------- elementwise warps 0..7
     const int h = warp >> 2;          // query half
     const int t = threadIdx.x & 127;  // key within the block == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int key = kblk * L::B + t;
     const float scale = p.scale;
     const float c_log2 = scale * kLog2e;
     const uint64_t C2 = f2_pack(c_log2, c_log2);
     const bool mode1 = p.mode == 1;
+    const int qoff = 64 * h;
+    const uint32_t ds_row = base + L::DS_OFF + h * TILE + t * 128;
+    BwdCursor cur;
+    cur.start(p);
+    int g = 0;
     bool ok = true;
-    for (int i = 0; i < n_it; ++i) {
-      const int b = i & 1;
-      if (!wait(bar(L::VEC_FULL + b), (i >> 1) & 1, 8)) { ok = false; break; }
-      if (!wait(bar(L::S_FULL + b), (i >> 1) & 1, 9)) { ok = false; break; }
-      if (threadIdx.x == 0) FA_TRACE_POINT(20);
-      tc_fence_after();
-      const uint32_t va = base + L::VEC_OFF + ((b * 3 + 0) * 128 + 64 * h) * 4;
-      const uint32_t vb = base + L::VEC_OFF + ((b * 3 + 1) * 128 + 64 * h) * 4;
-      const uint32_t vd = base + L::VEC_OFF + ((b * 3 + 2) * 128 + 64 * h) * 4;
-      const bool diag = p.causal && (i0 + i == kblk);
-      const int qoff = 64 * h;
-      uint64_t p2[32];  // this row's 64 P values (fp32 pairs)
-      {
-        uint32_t r0[32], r1[32];
-        tmem_ld32x2(tmem + lane_base + 128u * b + 64u * h, tmem + lane_base + 128u * b + 64u * h + 32u, r0, r1);
+    for (; ok && cur.valid; cur.next_item()) {
+      for (int i = 0; i < cur.n; ++i, ++g) {
+        const int b = g & 1;
+        if (!wait(bar(L::VEC_FULL + b), (g >> 1) & 1, 8)) { ok = false; break; }
+        if (!wait(bar(L::S_FULL + b), (g >> 1) & 1, 9)) { ok = false; break; }
+        if (threadIdx.x == 0) FA_TRACE_POINT(20);
+        tc_fence_after();
+        const uint32_t va = base + L::VEC_OFF + ((b * 3 + 0) * 128 + 64 * h) * 4;
+        const uint32_t vb = base + L::VEC_OFF + ((b * 3 + 1) * 128 + 64 * h) * 4;
+        const uint32_t vd = base + L::VEC_OFF + ((b * 3 + 2) * 128 + 64 * h) * 4;
+        const bool diag = p.causal && (cur.i0 + i == cur.kblk);
+        uint64_t p2[32];  // this row's 64 P values (fp32 pairs)
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32x2(tmem + lane_base + 128u * b + 64u * h, tmem + lane_base + 128u * b + 64u * h + 32u, r0, r1);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          p2[e] = f2_pack(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
-          p2[16 + e] = f2_pack(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+          for (int e = 0; e < 16; ++e) {
+            p2[e] = f2_pack(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
+            p2[16 + e] = f2_pack(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+          }
         }
-      }
-      if (threadIdx.x == 0) FA_TRACE_POINT(25);
-      // both warpgroups hold their S^T columns: P^T may now overwrite [0,64)
-      named_barrier_sync(1, 256);
-      if (threadIdx.x == 0) FA_TRACE_POINT(26);
-      uint32_t pk[32];
+        if (threadIdx.x == 0) FA_TRACE_POINT(25);
+        // both warpgroups hold their S^T columns: P^T may now overwrite [0,64)
+        named_barrier_sync(1, 256);
+        if (threadIdx.x == 0) FA_TRACE_POINT(26);
+        uint32_t pk[32];
 #pragma unroll
-      for (int pi = 0; pi < 32; pi += 2) {
-        const int ql = 2 * pi;
-        const float4 na = lds128(va + ql * 4);
-        const uint64_t y0 = f2_fma(p2[pi], C2, f2_pack(na.x, na.y));
-        const uint64_t y1 = f2_fma(p2[pi + 1], C2, f2_pack(na.z, na.w));
-        float a0, a1, a2, a3;
-        f2_unpack(y0, a0, a1);
-        f2_unpack(y1, a2, a3);
-        float p0 = ex2_approx(a0), p1 = ex2_approx(a1), p2v = ex2_approx(a2), p3 = ex2_approx(a3);
-        if (mode1) {
-          const float4 bb = lds128(vb + ql * 4);
-          p0 *= bb.x;
-          p1 *= bb.y;
-          p2v *= bb.z;
-          p3 *= bb.w;
+        for (int pi = 0; pi < 32; pi += 2) {
+          const int ql = 2 * pi;
+          const float4 na = lds128(va + ql * 4);
+          const uint64_t y0 = f2_fma(p2[pi], C2, f2_pack(na.x, na.y));
+          const uint64_t y1 = f2_fma(p2[pi + 1], C2, f2_pack(na.z, na.w));
+          float a0, a1, a2, a3;
+          f2_unpack(y0, a0, a1);
+          f2_unpack(y1, a2, a3);
+          float p0 = ex2_approx(a0), p1 = ex2_approx(a1), p2v = ex2_approx(a2), p3 = ex2_approx(a3);
+          if (mode1) {
+            const float4 bb = lds128(vb + ql * 4);
+            p0 *= bb.x;
+            p1 *= bb.y;
+            p2v *= bb.z;
+            p3 *= bb.w;
+          }
+          if (diag) {
+            const int qg = qoff + ql;
+            if (t > qg) p0 = 0.f;
+            if (t > qg + 1) p1 = 0.f;
+            if (t > qg + 2) p2v = 0.f;
+            if (t > qg + 3) p3 = 0.f;
+          }
+          p2[pi] = f2_pack(p0, p1);
+          p2[pi + 1] = f2_pack(p2v, p3);
+          pk[pi] = pack_bf16x2(p0, p1);
+          pk[pi + 1] = pack_bf16x2(p2v, p3);
         }
-        if (diag) {
-          const int qg = qoff + ql;
-          if (t > qg) p0 = 0.f;
-          if (t > qg + 1) p1 = 0.f;
-          if (t > qg + 2) p2v = 0.f;
-          if (t > qg + 3) p3 = 0.f;
+        tmem_st32(tmem + lane_base + 128u * b + 32u * h, pk);
+        if (threadIdx.x == 0) FA_TRACE_POINT(27);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::P_FULL + b));
+        if (threadIdx.x == 0) FA_TRACE_POINT(21);
+        if (!wait(bar(L::DP_FULL), g & 1, 10)) { ok = false; break; }
+        if (threadIdx.x == 0) FA_TRACE_POINT(22);
+        // the dQ product of the previous block has finished reading the dS tile
+        if (g > 0 && !wait(bar(L::DQ_FULL + ((g - 1) & 1)), ((g - 1) >> 1) & 1, 11)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t dpr[64];
+        {
+          uint32_t(&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]);
+          uint32_t(&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]);
+          tmem_ld32x2(tmem + lane_base + L::DPT_COL + 64u * h, tmem + lane_base + L::DPT_COL + 64u * h + 32u, d0,
+                      d1);
         }
-        p2[pi] = f2_pack(p0, p1);
-        p2[pi + 1] = f2_pack(p2v, p3);
-        pk[pi] = pack_bf16x2(p0, p1);
-        pk[pi + 1] = pack_bf16x2(p2v, p3);
-      }
-      tmem_st32(tmem + lane_base + 128u * b + 32u * h, pk);
-      if (threadIdx.x == 0) FA_TRACE_POINT(27);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(L::P_FULL + b));
-      if (threadIdx.x == 0) FA_TRACE_POINT(21);
-      if (!wait(bar(L::DP_FULL), i & 1, 10)) { ok = false; break; }
-      if (threadIdx.x == 0) FA_TRACE_POINT(22);
-      // the dQ product of the previous block has finished reading the dS tile
-      if (i > 0 && !wait(bar(L::DQ_FULL + ((i - 1) & 1)), ((i - 1) >> 1) & 1, 11)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t ds_row = base + L::DS_OFF + h * TILE + t * 128;
-      uint32_t dpr[64];
-      {
-        uint32_t (&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]);
-        uint32_t (&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]);
-        tmem_ld32x2(tmem + lane_base + L::DPT_COL + 64u * h, tmem + lane_base + L::DPT_COL + 64u * h + 32u, d0, d1);
-      }
-      uint32_t dk_[32];
+        uint32_t dk_[32];
 #pragma unroll
-      for (int pi = 0; pi < 32; pi += 2) {
-        const int ql = 2 * pi;
-        const float4 dl = lds128(vd + ql * 4);
-        const uint64_t ds0 = f2_mul(p2[pi], f2_sub(f2_pack(__uint_as_float(dpr[2 * pi]), __uint_as_float(dpr[2 * pi + 1])),
-                                                   f2_pack(dl.x, dl.y)));
-        const uint64_t ds1 = f2_mul(p2[pi + 1], f2_sub(f2_pack(__uint_as_float(dpr[2 * pi + 2]), __uint_as_float(dpr[2 * pi + 3])),
-                                                       f2_pack(dl.z, dl.w)));
-        float d0, d1, d2, d3;
-        f2_unpack(ds0, d0, d1);
-        f2_unpack(ds1, d2, d3);
-        dk_[pi] = pack_bf16x2(d0, d1);
-        dk_[pi + 1] = pack_bf16x2(d2, d3);
-      }
-      // dS^T into the dP^T columns this warpgroup has read: 64h + [0,32)
-      tmem_st32(tmem + lane_base + L::DPT_COL + 64u * h, dk_);
-      // dS^T row t, queries 64h + [0,64) = the eight 16-byte chunks of the half tile's row
+        for (int pi = 0; pi < 32; pi += 2) {
+          const int ql = 2 * pi;
+          const float4 dl = lds128(vd + ql * 4);
+          const uint64_t ds0 = f2_mul(
+              p2[pi], f2_sub(f2_pack(__uint_as_float(dpr[2 * pi]), __uint_as_float(dpr[2 * pi + 1])), f2_pack(dl.x, dl.y)));
+          const uint64_t ds1 =
+              f2_mul(p2[pi + 1], f2_sub(f2_pack(__uint_as_float(dpr[2 * pi + 2]), __uint_as_float(dpr[2 * pi + 3])),
+                                        f2_pack(dl.z, dl.w)));
+          float d0, d1, d2, d3;
+          f2_unpack(ds0, d0, d1);
+          f2_unpack(ds1, d2, d3);
+          dk_[pi] = pack_bf16x2(d0, d1);
+          dk_[pi + 1] = pack_bf16x2(d2, d3);
+        }
+        // dS^T into the dP^T columns this warpgroup has read: 64h + [0,32)
+        tmem_st32(tmem + lane_base + L::DPT_COL + 64u * h, dk_);
+        // dS^T row t, queries 64h + [0,64) = the eight 16-byte chunks of the half tile's row
 #pragma unroll
-      for (int chunk = 0; chunk < 8; ++chunk)
-        sts128(ds_row + ((chunk ^ (t & 7)) << 4), dk_[4 * chunk], dk_[4 * chunk + 1], dk_[4 * chunk + 2],
-               dk_[4 * chunk + 3]);
-      fence_proxy_async_smem();
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(L::DS_FULL));
-      mbar_arrive(bar(L::VEC_EMPTY + b));
-      if (threadIdx.x == 0) FA_TRACE_POINT(24);
-    }
-    // ------------------------------------------------------------- epilogue
-    // warpgroup 0 writes dV, warpgroup 1 writes dK * scale: TMEM -> bf16 rows
-    // in a 128B-swizzled tile (the dS tile, free once every product is done)
-    // -> one TMA tensor store per warpgroup (rows past N are clipped).
-    if (ok && wait(bar(L::ACC_DONE), 0, 12)) {
+        for (int chunk = 0; chunk < 8; ++chunk)
+          sts128(ds_row + ((chunk ^ (t & 7)) << 4), dk_[4 * chunk], dk_[4 * chunk + 1], dk_[4 * chunk + 2],
+                 dk_[4 * chunk + 3]);
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::DS_FULL));
+        mbar_arrive(bar(L::VEC_EMPTY + b));
+        if (threadIdx.x == 0) FA_TRACE_POINT(24);
+      }
+      if (!ok) break;
+      // ----------------------------------------------------- item epilogue
+      // warpgroup 0 writes dV, warpgroup 1 writes dK * scale: TMEM -> bf16
+      // rows in a 128B-swizzled tile (its half of the dS tile, whose last
+      // reader -- the item's final dQ product -- has completed) -> one TMA
+      // tensor store (rows past N are clipped).
+      if (!wait(bar(L::ACC_DONE), cur.r & 1, 12)) { ok = false; break; }
       tc_fence_after();
       const float f = (h == 0) ? 1.f : scale;
       const uint32_t col = (h == 0) ? L::DV_COL : L::DK_COL;
       uint32_t r0[32], r1[32];
       tmem_ld32x2(tmem + lane_base + col, tmem + lane_base + col + 32, r0, r1);
+      tc_fence_before();
+      mbar_arrive(bar(L::ACC_FREE));  // the next item may overwrite the accumulators
       uint32_t w[32];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
@@ -486,12 +578,13 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       named_barrier_sync(3 + h, 128);
       if (t == 0) {
         tma_store_3d(h == 0 ? static_cast<const void*>(&tm_dv) : static_cast<const void*>(&tm_dk),
-                     base + L::DS_OFF + h * TILE, 0, kblk * L::B, bh);
+                     base + L::DS_OFF + h * TILE, 0, cur.kblk * L::B, cur.bh);
         bulk_commit();
-        bulk_wait_all();
+        bulk_wait_read_all();  // the tile is the next item's dS tile
       }
+      named_barrier_sync(3 + h, 128);
     }
-    (void)key;
+    if (t == 0) bulk_wait_all();
     teardown();
   }
 }

@@ -257,12 +257,21 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_blk) * BH);
     if (D == 64) {
+      // persistent: one CTA per SM (at most one per work item)
+      static int n_sm = 0;
+      if (n_sm == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0)
+          return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)");
+      }
+      const unsigned pgrid = grid < static_cast<unsigned>(n_sm) ? grid : static_cast<unsigned>(n_sm);
       CUtensorMap mdq, mdk, mdv;
       if (!make_map_dq(&mdq, dq_acc, BH, N)) return cuda_fail("cuTensorMapEncodeTiled (dQ accumulator)");
       if (!make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
         return cuda_fail("cuTensorMapEncodeTiled (dk/dv)");
       LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
-      cudaError_t e = launch_pdl(fa::fa_bwd_main_pipe_kernel, dim3(grid), dim3(LP::THREADS), LP::SMEM_BYTES, stream,
+      cudaError_t e = launch_pdl(fa::fa_bwd_main_pipe_kernel, dim3(pgrid), dim3(LP::THREADS), LP::SMEM_BYTES, stream,
                                  mq, mk, mv, mdo, mdq, mdk, mdv, p);
       tm.done();
       if (e == cudaSuccess) e = cudaGetLastError();
