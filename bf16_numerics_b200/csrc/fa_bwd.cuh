@@ -347,20 +347,23 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     };
     float na, nb, nd;
     fetch(0, na, nb, nd);
+    // A bounded wait that gives up only clears `ok`; the four warps leave the
+    // loop together at the AND vote that opens the next iteration.
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int i = i0 + it;
       // publish this block's vectors (all 128 softmax threads), then prefetch the next
-      named_barrier_sync_128();
+      if (!named_barrier_and(1, 128, ok)) break;
       vec_a[t] = na;
       vec_b[t] = nb;
       vec_d[t] = nd;
       named_barrier_sync_128();
       fetch(it + 1, na, nb, nd);
       // dS smem is free once the previous dQ product has completed
-      if (it > 0 && !wait(bar(L::DQ_FULL), (it - 1) & 1, 8)) { ok = false; break; }
-      if (!wait(bar(L::S_FULL), it & 1, 9)) { ok = false; break; }
-      if (!wait(bar(L::DP_FULL), it & 1, 10)) { ok = false; break; }
+      ok = (it == 0 || wait.warp(bar(L::DQ_FULL), (it - 1) & 1, 8));
+      ok = ok && wait.warp(bar(L::S_FULL), it & 1, 9);
+      ok = ok && wait.warp(bar(L::DP_FULL), it & 1, 10);
+      if (!ok) continue;
       tc_fence_after();
       const bool diag = p.causal && (i == kblk);
 #pragma unroll 1
@@ -408,7 +411,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_arrive(bar(L::PDS_FULL));
     }
     // ------------------------------------------------------------- epilogue
-    if (ok && wait(bar(L::ACC_DONE), 0, 11)) {
+    if (ok && wait.warp(bar(L::ACC_DONE), 0, 11)) {
       tc_fence_after();
       const bool row_ok = key < p.N;
       __nv_bfloat16* dk_row = p.dk + (vrow0 + key) * D;

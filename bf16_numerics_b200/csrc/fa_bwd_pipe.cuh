@@ -384,10 +384,17 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     for (int k = 0; k < 2 && pub.valid; ++k, ++g_pub, pub.next_block()) publish_vec(g_pub, pub, load_vec(pub));
     Vec3 nxt = load_vec(pub);
     if (t == 0) tma_prefetch_desc(&tm_dq);
+    // A bounded wait that gives up only clears `ok`; the warpgroup leaves the
+    // loop together at the AND vote on named barrier 2 (a stale TMEM read
+    // before it is in bounds and harmless).
     bool ok = true;
-    for (int g = 0; ok && cur.valid; ++g, cur.next_block()) {
+    for (int g = 0; cur.valid; ++g, cur.next_block()) {
       const int b = g & 1;
-      if (!wait(bar(L::DQ_FULL + b), (g >> 1) & 1, 13)) break;
+      {
+        // every lane calls the warp-uniform wait (ok may differ per lane here)
+        const bool got = wait.warp(bar(L::DQ_FULL + b), (g >> 1) & 1, 13);
+        ok = ok && got;
+      }
       if (t == 0) FA_TRACE_POINT(30);
       tc_fence_after();
       uint32_t r0[32], r1[32];
@@ -395,7 +402,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       tc_fence_before();
       mbar_arrive(bar(L::DQ_FREE));
       if (t == 0) bulk_wait_read_all();  // the previous reduce has finished reading the staging tile
-      named_barrier_sync(2, 128);
+      if (!named_barrier_and(2, 128, ok)) break;
       // row t of each 32-column box, 16-byte chunk c stored at chunk c ^ (t & 7)
       const uint32_t row0 = base + L::DQS_OFF + t * 128;
       const uint32_t row1 = row0 + TILE;
@@ -422,11 +429,14 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       }
       if (pub.valid) {
         // block g+2 reuses the vector stage of block g
-        if (!wait(bar(L::VEC_EMPTY + b), (g >> 1) & 1, 14)) { ok = false; break; }
-        publish_vec(g_pub, pub, nxt);
-        ++g_pub;
-        pub.next_block();
-        nxt = load_vec(pub);
+        // (a wait that gives up skips the publish; the next vote ends the loop)
+        ok = wait(bar(L::VEC_EMPTY + b), (g >> 1) & 1, 14);
+        if (ok) {
+          publish_vec(g_pub, pub, nxt);
+          ++g_pub;
+          pub.next_block();
+          nxt = load_vec(pub);
+        }
       }
     }
     if (t == 0) bulk_wait_all();
@@ -449,12 +459,19 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     BwdCursor cur;
     cur.start(p);
     int g = 0;
+    // Error discipline: the two warpgroups meet on named barrier 1 once per
+    // block and once per item.  A bounded wait that gives up only clears `ok`
+    // (reads before the next meeting may see stale TMEM or shared memory,
+    // which is in bounds and harmless); each meeting is an AND vote, so both
+    // warpgroups leave together and neither is left waiting on a barrier the
+    // other no longer reaches.
     bool ok = true;
-    for (; ok && cur.valid; cur.next_item()) {
+    for (; cur.valid; cur.next_item()) {
+      bool leave = false;
       for (int i = 0; i < cur.n; ++i, ++g) {
         const int b = g & 1;
-        if (!wait(bar(L::VEC_FULL + b), (g >> 1) & 1, 8)) { ok = false; break; }
-        if (!wait(bar(L::S_FULL + b), (g >> 1) & 1, 9)) { ok = false; break; }
+        ok = ok && wait.warp(bar(L::VEC_FULL + b), (g >> 1) & 1, 8);
+        ok = ok && wait.warp(bar(L::S_FULL + b), (g >> 1) & 1, 9);
         if (threadIdx.x == 0) FA_TRACE_POINT(20);
         tc_fence_after();
         const uint32_t va = base + L::VEC_OFF + ((b * 3 + 0) * 128 + 64 * h) * 4;
@@ -473,7 +490,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         }
         if (threadIdx.x == 0) FA_TRACE_POINT(25);
         // both warpgroups hold their S^T columns: P^T may now overwrite [0,64)
-        named_barrier_sync(1, 256);
+        if (!named_barrier_and(1, 256, ok)) { leave = true; break; }
         if (threadIdx.x == 0) FA_TRACE_POINT(26);
         uint32_t pk[32];
 #pragma unroll
@@ -511,10 +528,11 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         tc_fence_before();
         mbar_arrive(bar(L::P_FULL + b));
         if (threadIdx.x == 0) FA_TRACE_POINT(21);
-        if (!wait(bar(L::DP_FULL), g & 1, 10)) { ok = false; break; }
+        ok = wait.warp(bar(L::DP_FULL), g & 1, 10);
         if (threadIdx.x == 0) FA_TRACE_POINT(22);
         // the dQ product of the previous block has finished reading the dS tile
-        if (g > 0 && !wait(bar(L::DQ_FULL + ((g - 1) & 1)), ((g - 1) >> 1) & 1, 11)) { ok = false; break; }
+        ok = ok && (g == 0 || wait.warp(bar(L::DQ_FULL + ((g - 1) & 1)), ((g - 1) >> 1) & 1, 11));
+        if (!ok) continue;  // the next meeting takes everyone out
         tc_fence_after();
         uint32_t dpr[64];
         {
@@ -553,13 +571,13 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         mbar_arrive(bar(L::VEC_EMPTY + b));
         if (threadIdx.x == 0) FA_TRACE_POINT(24);
       }
-      if (!ok) break;
+      if (leave) break;
       // ----------------------------------------------------- item epilogue
       // warpgroup 0 writes dV, warpgroup 1 writes dK * scale: TMEM -> bf16
       // rows in a 128B-swizzled tile (its half of the dS tile, whose last
       // reader -- the item's final dQ product -- has completed) -> one TMA
       // tensor store (rows past N are clipped).
-      if (!wait(bar(L::ACC_DONE), cur.r & 1, 12)) { ok = false; break; }
+      ok = ok && wait.warp(bar(L::ACC_DONE), cur.r & 1, 12);
       tc_fence_after();
       const float f = (h == 0) ? 1.f : scale;
       const uint32_t col = (h == 0) ? L::DV_COL : L::DK_COL;
@@ -575,7 +593,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       }
       sts_row_sw128(base + L::DS_OFF + h * TILE, t, w);
       fence_proxy_async_smem();
-      named_barrier_sync(3 + h, 128);
+      if (!named_barrier_and(1, 256, ok)) break;
       if (t == 0) {
         tma_store_3d(h == 0 ? static_cast<const void*>(&tm_dv) : static_cast<const void*>(&tm_dk),
                      base + L::DS_OFF + h * TILE, 0, cur.kblk * L::B, cur.bh);

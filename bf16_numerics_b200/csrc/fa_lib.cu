@@ -156,6 +156,19 @@ bool set_smem(K kernel, int bytes) {
   return true;
 }
 
+// Multiprocessor count of the current device (queried once per device).
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 bool shape_ok(int B, int H, int N, int d) {
   if (B < 0 || H < 0 || N < 0) return false;
   const long long BH = static_cast<long long>(B) * H;
@@ -179,7 +192,6 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
       !make_map(&mo, o, BH, N, D))
     return cuda_fail("cuTensorMapEncodeTiled (q/k/v/o)");
   fa::FwdParams p{};
-  p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   if (st) {
     p.st_rm = st->rm;
@@ -194,9 +206,14 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   p.mode = mode;
   p.beta = beta;
   p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
-  const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_qblk) * BH);
+  // persistent: CTAS_PER_SM CTAs per SM (at most one per work item)
+  const int n_sm = sm_count();
+  if (n_sm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)");
+  const long long items = static_cast<long long>(p.n_qblk) * BH;
+  const long long slots = static_cast<long long>(n_sm) * L::CTAS_PER_SM;
+  const unsigned grid = static_cast<unsigned>(items < slots ? items : slots);
   LaunchTimer tm(FA_KERNEL_FWD, stream);
-  cudaError_t e = launch_pdl(fa::fa_fwd_kernel<D>, dim3(grid), dim3(192), L::SMEM_BYTES, stream, mq, mk, mv, mo, p);
+  cudaError_t e = launch_pdl(fa::fa_fwd_kernel<D>, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, stream, mq, mk, mv, mo, p);
   tm.done();
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : cuda_fail("fa_fwd_kernel launch", e);
@@ -258,13 +275,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_blk) * BH);
     if (D == 64) {
       // persistent: one CTA per SM (at most one per work item)
-      static int n_sm = 0;
-      if (n_sm == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0)
-          return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)");
-      }
+      const int n_sm = sm_count();
+      if (n_sm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)");
       const unsigned pgrid = grid < static_cast<unsigned>(n_sm) ? grid : static_cast<unsigned>(n_sm);
       CUtensorMap mdq, mdk, mdv;
       if (!make_map_dq(&mdq, dq_acc, BH, N)) return cuda_fail("cuTensorMapEncodeTiled (dQ accumulator)");

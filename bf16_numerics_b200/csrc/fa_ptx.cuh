@@ -95,6 +95,11 @@ struct BoundedWait {
       }
     }
   }
+  // Warp-uniform form: true only if the wait succeeded in every lane, so the
+  // warp's .sync.aligned instructions after it see one decision.
+  __device__ __forceinline__ bool warp(uint32_t bar, uint32_t parity, uint32_t site) const {
+    return __all_sync(0xffffffffu, (*this)(bar, parity, site));
+  }
 };
 
 // Named barrier 1 over the first four warps (128 threads).
@@ -253,6 +258,22 @@ namespace fa {
 // Named barrier `id` over `count` threads (id 0 is __syncthreads).
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Named barrier that also ANDs a predicate over the participating threads:
+// every thread gets true only if every thread passed true.  Used where a group
+// of warps must take the same branch after a bounded wait (a wait that gave up
+// in one warp must make all of them skip the work and the later barriers).
+__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0u;
 }
 // global[dst] += shared[src] element-wise (fp32), `bytes` a multiple of 16,
 // both addresses 16-byte aligned; tracked by the issuing thread's bulk group.
