@@ -36,7 +36,8 @@ METRIC = "attention fwd+bwd TFLOP/s (causal) and % of B200 dense BF16 peak, stab
 WORKLOAD = "g2s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ("bf16_numerics_b200/csrc/fa_ptx.cuh", "bf16_numerics_b200/csrc/fa_fwd.cuh",
-                  "bf16_numerics_b200/csrc/fa_bwd.cuh", "bf16_numerics_b200/csrc/fa_lib.cu")
+                  "bf16_numerics_b200/csrc/fa_bwd.cuh", "bf16_numerics_b200/csrc/fa_bwd_pipe.cuh",
+                  "bf16_numerics_b200/csrc/fa_lib.cu")
 
 
 def parse_args():

@@ -39,27 +39,49 @@ namespace fa {
 // delta[r] = sum_c dO[r,c] * O[r,c] in fp32; also clears the dQ accumulator
 // row.
 // Memory bound: each row of O and dO is read once with 16-byte loads, LPR
-// lanes per row.
+// lanes per row; every warp takes U row groups at a time and issues all of
+// their loads before using any, so enough bytes are in flight to cover the
+// DRAM latency.
 template <int D>
 __global__ void __launch_bounds__(256)
 fa_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                     float* __restrict__ delta, float* __restrict__ dq_acc, long long rows) {
   constexpr int LPR = D / 8;               // lanes per row (8 bf16 per lane)
-  constexpr int RPW = 32 / LPR;            // rows per warp per step
+  constexpr int RPW = 32 / LPR;            // rows per warp per group
+  constexpr int U = 4;                     // row groups per warp per pass
   const int lane = threadIdx.x & 31;
   const long long warp_global = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const int sub = lane / LPR, li = lane % LPR;
   grid_launch_dependents();
   grid_dependency_wait();  // O comes from the forward grid
-  for (long long r0 = warp_global * RPW; r0 < rows; r0 += n_warps * RPW) {
-    const long long r = r0 + sub;
-    float acc = 0.f;
-    if (r < rows) {
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + r * D) + li);
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dO + r * D) + li);
-      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+  for (long long r0 = warp_global * (RPW * U); r0 < rows; r0 += n_warps * (RPW * U)) {
+    uint4 a[U], b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long r = r0 + u * RPW + sub;
+      if (r < rows) {
+        a[u] = __ldg(reinterpret_cast<const uint4*>(o + r * D) + li);
+        b[u] = __ldg(reinterpret_cast<const uint4*>(dO + r * D) + li);
+      } else {
+        a[u] = make_uint4(0u, 0u, 0u, 0u);
+        b[u] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long r = r0 + u * RPW + sub;
+      if (r < rows) {
+        float4* z = reinterpret_cast<float4*>(dq_acc + r * D) + 2 * li;
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
+      float acc = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 fa2 = __bfloat1622float2(pa[i]);
@@ -67,31 +89,46 @@ fa_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __
         acc = fmaf(fa2.x, fb2.x, acc);
         acc = fmaf(fa2.y, fb2.y, acc);
       }
-      float4* z = reinterpret_cast<float4*>(dq_acc + r * D) + 2 * li;
-      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
 #pragma unroll
-    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (r < rows && li == 0) delta[r] = acc;
+      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const long long r = r0 + u * RPW + sub;
+      if (r < rows && li == 0) delta[r] = acc;
+    }
   }
 }
 
 // --------------------------------------------------------------- dQ convert
+// dq = bf16(dq_acc), 8 values per thread and chunk, U chunks per thread per
+// pass with all loads issued first; the accumulator is dead afterwards, so
+// it is read with the streaming (evict-first) hint.
 __global__ void __launch_bounds__(256)
 fa_bwd_dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq, long long n8) {
+  constexpr int U = 4;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   grid_launch_dependents();
   grid_dependency_wait();  // the accumulator is complete once the main grid is
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(dq_acc) + 2 * i);
-    const float4 b = __ldg(reinterpret_cast<const float4*>(dq_acc) + 2 * i + 1);
-    uint4 w;
-    w.x = pack_bf16x2(a.x, a.y);
-    w.y = pack_bf16x2(a.z, a.w);
-    w.z = pack_bf16x2(b.x, b.y);
-    w.w = pack_bf16x2(b.z, b.w);
-    reinterpret_cast<uint4*>(dq)[i] = w;
+  for (long long i0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < n8; i0 += stride * U) {
+    float4 a[U], b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long i = i0 + u * stride;
+      if (i < n8) {
+        a[u] = __ldcs(reinterpret_cast<const float4*>(dq_acc) + 2 * i);
+        b[u] = __ldcs(reinterpret_cast<const float4*>(dq_acc) + 2 * i + 1);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long i = i0 + u * stride;
+      if (i < n8) {
+        uint4 w;
+        w.x = pack_bf16x2(a[u].x, a[u].y);
+        w.y = pack_bf16x2(a[u].z, a[u].w);
+        w.z = pack_bf16x2(b[u].x, b[u].y);
+        w.w = pack_bf16x2(b[u].z, b[u].w);
+        reinterpret_cast<uint4*>(dq)[i] = w;
+      }
+    }
   }
 }
 

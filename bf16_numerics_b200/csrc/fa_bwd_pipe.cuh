@@ -22,9 +22,10 @@
 //   * dQ_g = dS K is one N = 64 product into S^T cols [64,128) of the same
 //     buffer, which no later product of the block touches.
 //   * Four drain warps move the dQ partial from TMEM into a 128B-swizzled
-//     fp32 tile in shared memory and add it to the fp32 accumulator in global
-//     memory with one TMA tensor reduce-add per 32-column half (rows past N
-//     are clipped by the tensor map).  They also prepare the per-query
+//     fp32 staging box in shared memory and add it to the fp32 accumulator in
+//     global memory with one TMA tensor reduce-add per 32-column half, one
+//     half after the other through the same box (rows past N are clipped by
+//     the tensor map).  They also prepare the per-query
 //     vectors (lse or m, 1/l, delta) two blocks ahead.
 //
 // Barrier phases count a global query-block index g that runs across the
@@ -50,8 +51,8 @@ struct BwdPipeLayout {
   static constexpr int K_OFF = 0, V_OFF = TILE, Q_OFF = 2 * TILE;
   static constexpr int DO_OFF = Q_OFF + NST * TILE;
   static constexpr int DS_OFF = DO_OFF + NST * TILE;  // dS^T [keys][queries], two 64-query halves
-  static constexpr int DQS_OFF = DS_OFF + 2 * TILE;   // dQ staging: two [128 rows][32 fp32] swizzled boxes
-  static constexpr int VEC_OFF = DQS_OFF + 2 * TILE;  // [2 stages][3][128] fp32
+  static constexpr int DQS_OFF = DS_OFF + 2 * TILE;   // dQ staging: one [128 rows][32 fp32] swizzled box
+  static constexpr int VEC_OFF = DQS_OFF + TILE;      // [2 stages][3][128] fp32
   static constexpr int BAR_OFF = VEC_OFF + 2 * 3 * 128 * 4;
   enum {
     KV_FULL = 0,
@@ -403,30 +404,31 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       mbar_arrive(bar(L::DQ_FREE));
       if (t == 0) bulk_wait_read_all();  // the previous reduce has finished reading the staging tile
       if (!named_barrier_and(2, 128, ok)) break;
-      // row t of each 32-column box, 16-byte chunk c stored at chunk c ^ (t & 7)
-      const uint32_t row0 = base + L::DQS_OFF + t * 128;
-      const uint32_t row1 = row0 + TILE;
+      // row t of the 32-column box, 16-byte chunk c stored at chunk c ^ (t & 7);
+      // the two halves of the row go through the box one after the other
+      const uint32_t row = base + L::DQS_OFF + t * 128;
+      const int q0 = cur.qblk() * L::B;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t pc = (c ^ (t & 7)) << 4;
-        sts128(row0 + pc, __float_as_uint(__uint_as_float(r0[4 * c]) * scale),
-               __float_as_uint(__uint_as_float(r0[4 * c + 1]) * scale),
-               __float_as_uint(__uint_as_float(r0[4 * c + 2]) * scale),
-               __float_as_uint(__uint_as_float(r0[4 * c + 3]) * scale));
-        sts128(row1 + pc, __float_as_uint(__uint_as_float(r1[4 * c]) * scale),
-               __float_as_uint(__uint_as_float(r1[4 * c + 1]) * scale),
-               __float_as_uint(__uint_as_float(r1[4 * c + 2]) * scale),
-               __float_as_uint(__uint_as_float(r1[4 * c + 3]) * scale));
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t(&r)[32] = half == 0 ? r0 : r1;
+        if (half == 1) {
+          if (t == 0) bulk_wait_read_all();  // the first half's reduce has read the box
+          named_barrier_sync(2, 128);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          sts128(row + ((c ^ (t & 7)) << 4), __float_as_uint(__uint_as_float(r[4 * c]) * scale),
+                 __float_as_uint(__uint_as_float(r[4 * c + 1]) * scale),
+                 __float_as_uint(__uint_as_float(r[4 * c + 2]) * scale),
+                 __float_as_uint(__uint_as_float(r[4 * c + 3]) * scale));
+        fence_proxy_async_smem();
+        named_barrier_sync(2, 128);
+        if (t == 0) {
+          tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF, 32 * half, q0, cur.bh);
+          bulk_commit();
+        }
       }
-      fence_proxy_async_smem();
-      named_barrier_sync(2, 128);
-      if (t == 0) {
-        const int q0 = cur.qblk() * L::B;
-        tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF, 0, q0, cur.bh);
-        tma_reduce_add_3d(&tm_dq, base + L::DQS_OFF + TILE, 32, q0, cur.bh);
-        bulk_commit();
-        FA_TRACE_POINT(31);
-      }
+      if (t == 0) FA_TRACE_POINT(31);
       if (pub.valid) {
         // block g+2 reuses the vector stage of block g
         // (a wait that gives up skips the publish; the next vote ends the loop)

@@ -249,7 +249,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       !make_map(&mdo, dO, BH, N, D))
     return cuda_fail("cuTensorMapEncodeTiled (q/k/v/dO)");
   {
-    constexpr int rows_per_block = 8 * (32 / (D / 8));
+    constexpr int rows_per_block = 8 * (32 / (D / 8)) * 4;  // 8 warps x rows per group x 4 groups
     LaunchTimer tm(FA_KERNEL_BWD_DELTA, stream);
     cudaError_t e = launch_pdl(fa::fa_bwd_delta_kernel<D>, dim3(grid_for(rows, rows_per_block)), dim3(256), 0,
                                stream, static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO),
@@ -302,7 +302,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   {
     const long long n8 = rows * D / 8;
     LaunchTimer tm(FA_KERNEL_BWD_DQ, stream);
-    cudaError_t e = launch_pdl(fa::fa_bwd_dq_convert_kernel, dim3(grid_for(n8, 256)), dim3(256), 0, stream,
+    cudaError_t e = launch_pdl(fa::fa_bwd_dq_convert_kernel, dim3(grid_for(n8, 256 * 4)), dim3(256), 0, stream,
                                static_cast<const float*>(dq_acc), static_cast<__nv_bfloat16*>(dq), n8);
     tm.done();
     if (e == cudaSuccess) e = cudaGetLastError();
