@@ -167,6 +167,32 @@ def cpu_oracle_sample(w, mode, beta, seconds):
     return per_head * done, elapsed, done, threads
 
 
+# ------------------------------------------------------------------ ranks
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's copy of the workload: same shapes on every rank (weak
+    scaling), independent values."""
+    import workloads
+
+    return workloads.CONFIGS[WORKLOAD][5] + rank
+
+
+def rank_max(x: float, world: int, device=None) -> float:
+    """Max of x over all ranks (x itself on one rank)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world: int, flops_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
 def workload_config(w, mode, beta):
     return {"workload": f"{w.name}: GPT-2 small attention B{w.B} H{w.H} N{w.N} d{w.d} causal, "
                         f"{'stabilised' if mode == 1 else 'standard'} shift (beta={beta})",
@@ -216,7 +242,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = workloads.make(WORKLOAD, seed=workloads.CONFIGS[WORKLOAD][5] + rank)
+    w = workloads.make(WORKLOAD, seed=rank_seed(rank))
     B, H, N, d = w.B, w.H, w.N, w.d
     mode, beta, causal = args.mode, args.beta, w.causal
 
@@ -271,11 +297,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     clocks = sampler.stop()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, stops)]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms_max = float(t.item())
+    total_ms_max = rank_max(sum(step_ms), world, dev)
     # per-kernel durations: a second timed pass with the library recording
     # CUDA events on the launching stream around each of its launches
     KR = min(K, 200)
@@ -291,7 +313,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device error word {word:#x} during timing")
 
     flops_step = w.flops_total()
-    value = world * flops_step * K / (total_ms_max * 1e-3) / 1e12
+    value = aggregate_tflops(world, flops_step, K, total_ms_max)
 
     # -------- end to end through the public API with host buffers
     E = args.e2e_steps
@@ -317,10 +339,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * flops_step * E / (float(te.item()) * 1e-3) / 1e12
+    e2e_value = aggregate_tflops(world, flops_step, E, rank_max(e0.elapsed_time(e1), world, dev))
 
     if rank != 0:
         return 0
