@@ -36,8 +36,15 @@ Readings where the pages are silent (each listed in the design notes):
   with S = (Q K^T) * scale in float64.  Where Q K^T is exact in binary32 and
   scale is a power of two (d = 64) the two coincide.
 * The backward's softmax recompute follows the mode switch: mode 0 uses
-  P = exp(S - lse); mode 1 rebuilds P_bar = exp(S - m) and P = P_bar * (1/l)
-  with l = exp(lse - m).  Both equal softmax(S) in exact arithmetic.
+  P = exp(S - lse); modes 1 and 2 rebuild P_bar = exp(S - m) and
+  P = P_bar * (1/l) with l = exp(lse - m).  All equal softmax(S) in exact
+  arithmetic.
+* Mode 2 (margin variant, the pages' fix carried to the bf16 operand): the
+  rule keeps max(P_bar) < 1 in fp32, but bf16(P_bar) still rounds to 1.0
+  when m - rm < 2^-9.  Mode 2 takes mode 1's m and, on tied rows where
+  m - rm < 2^-8 (binary32 subtraction), uses m = rm + 2^-8 (binary32 add)
+  instead, so exp(rm - m) <= exp(-2^-8) < 1 - 2^-9 and its bf16 value is
+  below 1 as well.
 * Causal masking: key j is visible to query i iff j <= i (equal lengths).
 """
 
@@ -47,6 +54,8 @@ import numpy as np
 
 STANDARD = 0
 STABILIZED = 1
+STABILIZED_MARGIN = 2
+MARGIN = np.float32(2.0 ** -8)  # mode 2: minimum m - rm on tied rows
 
 
 def scale_f64(d: int) -> float:
@@ -60,7 +69,8 @@ def scale_f32(d: int) -> np.float32:
 def select_shift(rm, rs, beta: float, mode: int = STABILIZED) -> np.ndarray:
     """Row shift m from the row max rm and tie count rs ("minimal fix" rule).
 
-    Evaluated in binary32 (beta*rm is a binary32 product).  Mode 0 returns rm.
+    Evaluated in binary32 (beta*rm is a binary32 product).  Mode 0 returns rm;
+    mode 2 applies the margin of the module docstring on top of mode 1.
     """
     rm = np.asarray(rm, dtype=np.float32)
     rs = np.asarray(rs)
@@ -72,8 +82,11 @@ def select_shift(rm, rs, beta: float, mode: int = STABILIZED) -> np.ndarray:
     zero_case = np.float32(b - np.float32(1.0))
     m = np.where(tied & (rm > 0), pos,
                  np.where(tied & (rm < 0), np.float32(0.0),
-                          np.where(tied & (rm == 0), zero_case, rm)))
-    return m.astype(np.float32)
+                          np.where(tied & (rm == 0), zero_case, rm))).astype(np.float32)
+    if mode == STABILIZED_MARGIN:
+        gap = (m - rm).astype(np.float32)
+        m = np.where(tied & (gap < MARGIN), (rm + MARGIN).astype(np.float32), m).astype(np.float32)
+    return m
 
 
 def _mask(n: int, causal: bool) -> np.ndarray:

@@ -19,6 +19,7 @@ import torch
 
 import workloads
 from oracle import attention as A
+from oracle import bf16
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -273,6 +274,61 @@ def test_o_for_delta_changes_only_delta_path():
 
 
 # ------------------------------------------------------- planted mistakes
+
+# ------------------------------------------------ margin variant (mode 2)
+
+def _small_tie_rows():
+    """One head of d = 64 on the 1/8 grid in which every row has a tied
+    maximum rm = 2^-9: q = +-e_i / 8; keys 0, 1 are (1/8) on dims 0-3 and the
+    other keys -(1/8) there, so even rows tie on keys 0, 1 and odd rows on the
+    other fourteen (S = +-2^-9)."""
+    N, d = 16, 64
+    q = np.zeros((1, 1, N, d), np.float32)
+    k = np.zeros((1, 1, N, d), np.float32)
+    v = workloads.to_bf16_values(np.random.default_rng(3).standard_normal((1, 1, N, d)).astype(np.float32))
+    for i in range(N):
+        q[0, 0, i, i % 4] = 0.125 if i % 2 == 0 else -0.125
+    for j in (0, 1):
+        k[0, 0, j, :4] = 0.125                    # tie pair for every query
+    k[0, 0, 2:, :4] = -0.125
+    return q, k, v
+
+
+def test_margin_keeps_bf16_pbar_below_one():
+    """Reading of the pages' goal max(P_bar) < 1 for the bf16 operand: with
+    |rm| = 2^-9 the fp32 rule leaves exp(rm - m) within 2^-9 of 1, which
+    rounds to 1.0 in bf16; the margin mode moves m by 2^-8 and the bf16 value
+    stays below 1.  (Closed form: bf16(exp(-2^-8)) = 1 - 2^-8.)"""
+    q, k, v = _small_tie_rows()
+    f1 = A.attention_fwd(q, k, v, False, 1)
+    f2 = A.attention_fwd(q, k, v, False, 2)
+    tied = f1["rs"] > 1
+    assert tied.all() and np.all(f1["rm"] == np.float32(2.0 ** -9))
+    bf1 = bf16.round_bf16(f1["pbar_max"].astype(np.float32))
+    bf2 = bf16.round_bf16(f2["pbar_max"].astype(np.float32))
+    assert np.all(f1["pbar_max"][tied] < 1.0)          # the fp32 rule holds ...
+    assert np.all(bf1[tied] == 1.0)                    # ... but its bf16 value is 1
+    assert np.all(bf2[tied] < 1.0)
+    assert np.all(bf2[tied] <= np.float32(1.0 - 2.0 ** -8))
+    assert np.all(f2["m"][~tied] == f2["rm"][~tied])
+    # the margin is a shift: O and lse are unchanged (softmax shift invariance)
+    np.testing.assert_allclose(f2["o"], f1["o"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(f2["lse"], f1["lse"], rtol=1e-12)
+
+
+def test_margin_sweep_over_tied_maxima():
+    """Every tied row, whatever rm, ends with bf16(exp(rm - m)) < 1 in mode 2."""
+    rng = np.random.default_rng(5)
+    rm = np.concatenate([rng.uniform(-1e-2, 1e-2, 20000), rng.uniform(-50, 50, 20000),
+                         np.array([0.0, 2.0 ** -9, -(2.0 ** -9), 2.0 ** -8, -(2.0 ** -8)])]).astype(np.float32)
+    rs = np.full(rm.shape, 2)
+    for beta in (1.001, 1.5, 2.0, 4.0):
+        m = A.select_shift(rm, rs, beta, 2)
+        assert np.all((m - rm).astype(np.float32) >= np.float32(2.0 ** -8) * np.float32(0.999))
+        pmax = np.exp(rm.astype(np.float64) - m.astype(np.float64)).astype(np.float32)
+        ok = np.isfinite(pmax) & (pmax > 0)
+        assert np.all(bf16.round_bf16(pmax[ok]) < 1.0)
+
 
 def test_planted_mistake_dropped_scale_is_caught(monkeypatch):
     monkeypatch.setattr(A, "scale_f64", lambda d: 1.0)
