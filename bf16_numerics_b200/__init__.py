@@ -24,8 +24,9 @@ from . import _abi
 
 STANDARD = _abi.FA_SOFTMAX_STANDARD
 STABILIZED = _abi.FA_SOFTMAX_STABILIZED
+STABILIZED_MARGIN = _abi.FA_SOFTMAX_STABILIZED_MARGIN
 
-__all__ = ["FaError", "STANDARD", "STABILIZED", "RowStats", "fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes",
+__all__ = ["FaError", "STANDARD", "STABILIZED", "STABILIZED_MARGIN", "RowStats", "fa_fwd", "fa_bwd", "fa_fwd_o_hp", "fa_bwd_o_hp", "fa_bwd_workspace_bytes",
            "fa_bwd_workspace_offsets", "fa_status_string", "fa_device_error", "fa_timing_enable",
            "fa_timing_read", "attention_forward", "attention_backward", "library_path"]
 
@@ -87,6 +88,19 @@ def fa_status_string(code: int) -> str:
     return _abi.status_string(code)
 
 
+def _stats_struct(stats, B, H, N):
+    if stats is None:
+        return None
+    for name in ("rm", "m", "pbar_max"):
+        t = getattr(stats, name)
+        if t is not None:
+            _check_vec(f"stats.{name}", t, (B, H, N))
+    if stats.rs is not None:
+        _check_vec("stats.rs", stats.rs, (B, H, N), torch.int32)
+    return _abi.FaRowStats(*(None if getattr(stats, n) is None else getattr(stats, n).data_ptr()
+                             for n in ("rm", "rs", "m", "pbar_max")))
+
+
 def fa_fwd(q, k, v, o, lse, stats: RowStats | None = None, causal: bool = True, softmax_mode: int = STABILIZED,
            beta: float = 2.0, stream=None) -> None:
     """C ``fa_fwd``: writes o (bf16) and lse (fp32 [B,H,N]) and, if given, the row stats."""
@@ -96,20 +110,29 @@ def fa_fwd(q, k, v, o, lse, stats: RowStats | None = None, causal: bool = True, 
     for name, t in (("k", k), ("v", v), ("o", o)):
         _check_qkv(name, t, q.shape)
     _check_vec("lse", lse, (B, H, N))
-    st = None
-    if stats is not None:
-        for name in ("rm", "m", "pbar_max"):
-            t = getattr(stats, name)
-            if t is not None:
-                _check_vec(f"stats.{name}", t, (B, H, N))
-        if stats.rs is not None:
-            _check_vec("stats.rs", stats.rs, (B, H, N), torch.int32)
-        st = _abi.FaRowStats(*(None if getattr(stats, n) is None else getattr(stats, n).data_ptr()
-                               for n in ("rm", "rs", "m", "pbar_max")))
+    st = _stats_struct(stats, B, H, N)
     code = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(st) if st is not None else None,
                       B, H, N, d, int(bool(causal)), int(softmax_mode), float(beta), _stream_handle(stream))
     if code != _abi.FA_OK:
         raise FaError(code, "fa_fwd")
+
+
+def fa_fwd_o_hp(q, k, v, o, o_hp, lse, stats: RowStats | None = None, causal: bool = True,
+                softmax_mode: int = STABILIZED, beta: float = 2.0, stream=None) -> None:
+    """C ``fa_fwd_o_hp``: fa_fwd plus the fp32 O before rounding (o_hp, fp32 [B,H,N,d])."""
+    lib = _abi.load()
+    _check_qkv("q", q)
+    B, H, N, d = q.shape
+    for name, t in (("k", k), ("v", v), ("o", o)):
+        _check_qkv(name, t, q.shape)
+    _check_vec("o_hp", o_hp, (B, H, N, d))
+    _check_vec("lse", lse, (B, H, N))
+    st = _stats_struct(stats, B, H, N)
+    code = lib.fa_fwd_o_hp(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(o_hp), _ptr(lse),
+                           ctypes.byref(st) if st is not None else None, B, H, N, d, int(bool(causal)),
+                           int(softmax_mode), float(beta), _stream_handle(stream))
+    if code != _abi.FA_OK:
+        raise FaError(code, "fa_fwd_o_hp")
 
 
 def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
@@ -121,24 +144,43 @@ def fa_bwd_workspace_offsets(B: int, H: int, N: int, d: int) -> tuple[int, int]:
     return int(lib.fa_bwd_workspace_delta_offset(B, H, N, d)), int(lib.fa_bwd_workspace_dq_offset(B, H, N, d))
 
 
-def fa_bwd(q, k, v, o, dO, lse, row_m, dq, dk, dv, workspace, causal: bool = True, softmax_mode: int = STABILIZED,
-           beta: float = 2.0, stream=None) -> None:
-    """C ``fa_bwd``: writes dq, dk, dv (bf16); workspace is a uint8 CUDA tensor."""
-    lib = _abi.load()
+def _bwd_checks(q, k, v, dO, lse, row_m, dq, dk, dv, workspace):
     _check_qkv("q", q)
     B, H, N, d = q.shape
-    for name, t in (("k", k), ("v", v), ("o", o), ("dO", dO), ("dq", dq), ("dk", dk), ("dv", dv)):
+    for name, t in (("k", k), ("v", v), ("dO", dO), ("dq", dq), ("dk", dk), ("dv", dv)):
         _check_qkv(name, t, q.shape)
     _check_vec("lse", lse, (B, H, N))
     if row_m is not None:
         _check_vec("row_m", row_m, (B, H, N))
     if workspace.dtype != torch.uint8 or not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
+    return B, H, N, d
+
+
+def fa_bwd(q, k, v, o, dO, lse, row_m, dq, dk, dv, workspace, causal: bool = True, softmax_mode: int = STABILIZED,
+           beta: float = 2.0, stream=None) -> None:
+    """C ``fa_bwd``: writes dq, dk, dv (bf16); workspace is a uint8 CUDA tensor."""
+    lib = _abi.load()
+    B, H, N, d = _bwd_checks(q, k, v, dO, lse, row_m, dq, dk, dv, workspace)
+    _check_qkv("o", o, q.shape)
     code = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(row_m), _ptr(dq), _ptr(dk),
                       _ptr(dv), _ptr(workspace), workspace.numel(), B, H, N, d, int(bool(causal)),
                       int(softmax_mode), float(beta), _stream_handle(stream))
     if code != _abi.FA_OK:
         raise FaError(code, "fa_bwd")
+
+
+def fa_bwd_o_hp(q, k, v, o_hp, dO, lse, row_m, dq, dk, dv, workspace, causal: bool = True,
+                softmax_mode: int = STABILIZED, beta: float = 2.0, stream=None) -> None:
+    """C ``fa_bwd_o_hp``: fa_bwd with delta taken from the fp32 O (o_hp, fp32 [B,H,N,d])."""
+    lib = _abi.load()
+    B, H, N, d = _bwd_checks(q, k, v, dO, lse, row_m, dq, dk, dv, workspace)
+    _check_vec("o_hp", o_hp, (B, H, N, d))
+    code = lib.fa_bwd_o_hp(_ptr(q), _ptr(k), _ptr(v), _ptr(o_hp), _ptr(dO), _ptr(lse), _ptr(row_m), _ptr(dq),
+                           _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), B, H, N, d, int(bool(causal)),
+                           int(softmax_mode), float(beta), _stream_handle(stream))
+    if code != _abi.FA_OK:
+        raise FaError(code, "fa_bwd_o_hp")
 
 
 def fa_device_error() -> tuple[int, int]:

@@ -20,6 +20,7 @@ FA_ERR_TIMEOUT = 5
 
 FA_SOFTMAX_STANDARD = 0
 FA_SOFTMAX_STABILIZED = 1
+FA_SOFTMAX_STABILIZED_MARGIN = 2
 
 FA_KERNEL_FWD = 0
 FA_KERNEL_BWD_DELTA = 1
@@ -31,7 +32,7 @@ KERNEL_NAMES = ("fa_fwd_kernel", "fa_bwd_delta_kernel", "fa_bwd_main_kernel", "f
 # every symbol include/fa_b200.h declares
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_workspace_delta_offset",
            "fa_bwd_workspace_dq_offset", "fa_status_string", "fa_device_error", "fa_timing_enable",
-           "fa_timing_read", "fa_bwd_noalloc", "fa_last_error_string")
+           "fa_timing_read", "fa_bwd_noalloc", "fa_last_error_string", "fa_fwd_o_hp", "fa_bwd_o_hp")
 
 
 class FaRowStats(ctypes.Structure):
@@ -54,6 +55,10 @@ def load() -> ctypes.CDLL:
     lib.fa_fwd.restype = i
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, f, vp]
     lib.fa_bwd.restype = i
+    lib.fa_fwd_o_hp.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(FaRowStats), i, i, i, i, i, i, f, vp]
+    lib.fa_fwd_o_hp.restype = i
+    lib.fa_bwd_o_hp.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, f, vp]
+    lib.fa_bwd_o_hp.restype = i
     for name in ("fa_bwd_workspace_bytes", "fa_bwd_workspace_delta_offset", "fa_bwd_workspace_dq_offset"):
         getattr(lib, name).argtypes = [i, i, i, i]
         getattr(lib, name).restype = sz

@@ -37,16 +37,34 @@ namespace fa {
 
 // ------------------------------------------------------------------ delta
 // delta[r] = sum_c dO[r,c] * O[r,c] in fp32; also clears the dQ accumulator
-// row.
+// row.  O is the bf16 output of the forward, or (OT = float) its fp32 value
+// before rounding (the high-precision O_hp of the pages).
 // Memory bound: each row of O and dO is read once with 16-byte loads, LPR
-// lanes per row; every warp takes U row groups at a time and issues all of
-// their loads before using any, so enough bytes are in flight to cover the
-// DRAM latency.
-template <int D>
+// lanes per row (8 elements of dO per lane); every warp takes U row groups at
+// a time and issues all of their loads before using any, so enough bytes are
+// in flight to cover the DRAM latency.
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __bfloat1622float2(pa[i]);
+    f[2 * i] = x.x;
+    f[2 * i + 1] = x.y;
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+template <int D, typename OT>
 __global__ void __launch_bounds__(256)
-fa_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                     float* __restrict__ delta, float* __restrict__ dq_acc, long long rows) {
-  constexpr int LPR = D / 8;               // lanes per row (8 bf16 per lane)
+  constexpr int LPR = D / 8;               // lanes per row (8 elements per lane)
   constexpr int RPW = 32 / LPR;            // rows per warp per group
   constexpr int U = 4;                     // row groups per warp per pass
   const int lane = threadIdx.x & 31;
@@ -56,16 +74,16 @@ fa_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __
   grid_launch_dependents();
   grid_dependency_wait();  // O comes from the forward grid
   for (long long r0 = warp_global * (RPW * U); r0 < rows; r0 += n_warps * (RPW * U)) {
-    uint4 a[U], b[U];
+    float a[U][8], b[U][8];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const long long r = r0 + u * RPW + sub;
       if (r < rows) {
-        a[u] = __ldg(reinterpret_cast<const uint4*>(o + r * D) + li);
-        b[u] = __ldg(reinterpret_cast<const uint4*>(dO + r * D) + li);
+        load8(o + r * D + 8 * li, a[u]);
+        load8(dO + r * D + 8 * li, b[u]);
       } else {
-        a[u] = make_uint4(0u, 0u, 0u, 0u);
-        b[u] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[u][i] = b[u][i] = 0.f;
       }
     }
 #pragma unroll
@@ -79,16 +97,9 @@ fa_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
-      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
       float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 fa2 = __bfloat1622float2(pa[i]);
-        const float2 fb2 = __bfloat1622float2(pb[i]);
-        acc = fmaf(fa2.x, fb2.x, acc);
-        acc = fmaf(fa2.y, fb2.y, acc);
-      }
+      for (int i = 0; i < 8; ++i) acc = fmaf(a[u][i], b[u][i], acc);
 #pragma unroll
       for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
       const long long r = r0 + u * RPW + sub;

@@ -4,6 +4,7 @@
 // "mechanism two" and "minimal fix"):
 //   S = Q K^T * scale, rm = rowmax(S), rs = rowsum(S == rm),
 //   m = beta*rm (rs>1, rm>0) | 0 (rs>1, rm<0) | beta-1 (rs>1, rm==0) | rm,
+//   and in the margin mode, on tied rows, m = rm + 2^-8 where m - rm < 2^-8,
 //   P_bar = exp(S - m), P = P_bar / rowsum(P_bar), O = P V, lse = m + ln(l).
 // The row statistics are kept online across key tiles: a later tile with a
 // larger maximum resets (rm, rs); an equal maximum adds its tie count; whenever
@@ -53,9 +54,13 @@
 namespace fa {
 
 constexpr float kLog2e = 1.4426950408889634f;
+// margin mode: minimum m - rm on rows with a tied maximum (2^-8), so that
+// bf16(exp(rm - m)) < 1 as well
+constexpr float kShiftMargin = 0.00390625f;
 
 struct FwdParams {
   float* lse;         // [BH, N]
+  float* o_hp;        // optional fp32 O [BH, N, D] (the normalised accumulator before bf16 rounding)
   float* st_rm;       // optional [BH, N]
   int32_t* st_rs;     // optional
   float* st_m;        // optional
@@ -65,7 +70,7 @@ struct FwdParams {
   float beta, scale;
 };
 
-template <int D>
+template <int D, bool HP = false>
 struct FwdLayout {
   static constexpr int BM = 128, BN = 128;
   static constexpr int TILE = BM * D * 2;  // bytes of a 128 x D bf16 tile
@@ -82,8 +87,12 @@ struct FwdLayout {
   };
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base (4B), abort flag (4B)
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
-  static constexpr uint32_t S_COL = 0, P_COL = 128, O_COL = 192;
-  static constexpr uint32_t TMEM_COLS = (O_COL + D <= 256) ? 256 : 512;
+  // HP (high-precision O requested): P_bar also as a second bf16 part
+  // P_lo = bf16(P_bar - P_hi) at PLO_COL, multiplied into its own
+  // accumulator O_lo, so that (O + O_lo) / l carries P_bar to ~16 bits
+  static constexpr uint32_t S_COL = 0, P_COL = 128, PLO_COL = 192;
+  static constexpr uint32_t O_COL = HP ? 256 : 192, OLO_COL = 256 + D;
+  static constexpr uint32_t TMEM_COLS = (!HP && O_COL + D <= 256) ? 256 : 512;
   static constexpr int CTAS_PER_SM = (TMEM_COLS == 256) ? 2 : 1;
   static constexpr int THREADS = 384;
   // register budgets after setmaxnreg (two CTAs per SM: 80 per thread at
@@ -124,12 +133,12 @@ struct FwdCursor {
   __device__ __forceinline__ bool has_next(const FwdParams& p) const { return item(r + 1) < p.n_qblk * p.BH; }
 };
 
-template <int D>
-__global__ void __launch_bounds__(384, FwdLayout<D>::CTAS_PER_SM)
+template <int D, bool HP>
+__global__ void __launch_bounds__(384, FwdLayout<D, HP>::CTAS_PER_SM)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
               const FwdParams p) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, HP>;
   constexpr bool kRawCompare = (D == 64);  // scale is exactly 1/8
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -323,6 +332,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const uint64_t b = sdesc_sw128(vbase + ks * 2048, L::HALF, 1024);
             mma_ts(tmem + L::O_COL, tmem + L::P_COL + 8u * ks, b, IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
           }
+          if constexpr (HP) {
+#pragma unroll
+            for (int ks = 0; ks < L::BN / 16; ++ks) {
+              const uint64_t b = sdesc_sw128(vbase + ks * 2048, L::HALF, 1024);
+              mma_ts(tmem + L::OLO_COL, tmem + L::PLO_COL + 8u * ks, b, IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
+            }
+          }
           tc_commit(bar(L::O_READY));
           tc_commit(bar(L::V_EMPTY + (gt & 1)));
           FA_TRACE_POINT(11);
@@ -442,7 +458,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         const float rm_s = rm_x * to_s;
         float m_new = rm_s;
-        if (p.mode == 1 && rs > 1) m_new = (rm_s > 0.f) ? beta * rm_s : ((rm_s < 0.f) ? 0.f : beta - 1.f);
+        if (p.mode != 0 && rs > 1) {
+          // binary32 operations without contraction, as the rule states them
+          m_new = (rm_s > 0.f) ? __fmul_rn(beta, rm_s) : ((rm_s < 0.f) ? 0.f : __fsub_rn(beta, 1.f));
+          if (p.mode == 2 && __fsub_rn(m_new, rm_s) < kShiftMargin) m_new = __fadd_rn(rm_s, kShiftMargin);
+        }
         if (threadIdx.x == 0) FA_TRACE_POINT(22);
         // P_bar = exp2(x * exp_c - m * log2e) for this half, packed to bf16 pairs
         // in registers (the TMEM P slot is still being read by the previous P V
@@ -451,6 +471,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint64_t NM2 = f2_pack(nm, nm);
         uint64_t sum2[2] = {0ull, 0ull};
         uint32_t pk[32];
+        uint32_t plo[HP ? 32 : 1];  // HP: P_bar - bf16(P_bar), rounded to bf16
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const uint64_t y = f2_fma(f2_pack(x[c], x[c + 1]), EXPC2, NM2);
@@ -459,6 +480,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           const float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
           sum2[(c >> 1) & 1] = f2_add(sum2[(c >> 1) & 1], f2_pack(e0, e1));
           pk[c >> 1] = pack_bf16x2(e0, e1);
+          if constexpr (HP) {
+            const float h0 = __uint_as_float(pk[c >> 1] << 16), h1 = __uint_as_float(pk[c >> 1] & 0xffff0000u);
+            plo[c >> 1] = pack_bf16x2(e0 - h0, e1 - h1);
+          }
         }
         float psum;
         {
@@ -476,6 +501,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           tc_fence_after();
         }
         tmem_st32(tmem + lane_base + L::P_COL + 32u * h, pk);
+        if constexpr (HP) tmem_st32(tmem + lane_base + L::PLO_COL + 32u * h, plo);
         if (j > 0) {
           const bool changed = (m_new != m_run);
           float alpha = 1.f;
@@ -485,9 +511,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           }
           if (__any_sync(0xffffffffu, changed)) {
 #pragma unroll 1
-            for (int c0 = 0; c0 < DH; c0 += 16) {
+            for (int c0 = 0; c0 < (HP ? 2 * DH : DH); c0 += 16) {
               uint32_t r[16];
-              const uint32_t oa = tmem + lane_base + L::O_COL + DH * h + c0;
+              const uint32_t acc_col = (c0 < DH) ? (L::O_COL + c0) : (L::OLO_COL + c0 - DH);
+              const uint32_t oa = tmem + lane_base + acc_col + DH * h;
               tmem_ld16(oa, r);
 #pragma unroll
               for (int c = 0; c < 16; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
@@ -521,10 +548,29 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const float lsum = l + lo;
       const float inv_l = 1.f / lsum;
       // this half's O columns -> bf16 -> the item's Q buffer, 128B-swizzled
+      // (and, if asked, the same fp32 values to o_hp)
       const uint32_t stage = base + L::Q_OFF + (cur.r & 1) * L::TILE;
+      const int q_row = qblk * L::BM + t;
+      // o_hp (HP only) = (O + O_lo) / l; the bf16 o is fa_fwd's, from O alone
+      float* hp_row = (HP && q_row < p.N) ? p.o_hp + (static_cast<size_t>(cur.bh) * p.N + q_row) * D + DH * h
+                                           : nullptr;
+      auto write_hp = [&](float* dst, const uint32_t (&o_)[32], uint32_t lo_col) {
+        uint32_t lo[32];
+        tmem_ld32(lo_col, lo);
+        if (dst) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(dst + c) = make_float4(
+                (__uint_as_float(o_[c]) + __uint_as_float(lo[c])) * inv_l,
+                (__uint_as_float(o_[c + 1]) + __uint_as_float(lo[c + 1])) * inv_l,
+                (__uint_as_float(o_[c + 2]) + __uint_as_float(lo[c + 2])) * inv_l,
+                (__uint_as_float(o_[c + 3]) + __uint_as_float(lo[c + 3])) * inv_l);
+        }
+      };
       if constexpr (D == 64) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_base + L::O_COL + 32u * h, r);
+        if constexpr (HP) write_hp(hp_row, r, tmem + lane_base + L::OLO_COL + 32u * h);
         const uint32_t rp = stage + t * 128;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -538,6 +584,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       } else {
         uint32_t r0[32], r1[32];
         tmem_ld32x2(tmem + lane_base + L::O_COL + 64u * h, tmem + lane_base + L::O_COL + 64u * h + 32, r0, r1);
+        if constexpr (HP) {
+          write_hp(hp_row, r0, tmem + lane_base + L::OLO_COL + 64u * h);
+          write_hp(hp_row ? hp_row + 32 : nullptr, r1, tmem + lane_base + L::OLO_COL + 64u * h + 32);
+        }
         uint32_t w[32];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -549,7 +599,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       fence_proxy_async_smem();
       mbar_arrive(bar(L::O_STAGED + (cur.r & 1)));
       if (threadIdx.x == 0) FA_TRACE_POINT(25);
-      const int q_row = qblk * L::BM + t;
       if (h == 0 && q_row < p.N) {
         const size_t ri = static_cast<size_t>(cur.bh) * p.N + q_row;
         const float rm_s = rm_x * to_s;

@@ -179,20 +179,15 @@ bool shape_ok(int B, int H, int N, int d) {
 }
 
 template <int D>
-fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const fa_row_stats* st,
-                     int BH, int N, int causal, int mode, float beta, cudaStream_t stream) {
-  using L = fa::FwdLayout<D>;
-  static bool attr = false;
-  if (!attr) {
-    if (!set_smem(fa::fa_fwd_kernel<D>, L::SMEM_BYTES)) return FA_ERR_CUDA;
-    attr = true;
-  }
+fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* o_hp, float* lse,
+                     const fa_row_stats* st, int BH, int N, int causal, int mode, float beta, cudaStream_t stream) {
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D) ||
       !make_map(&mo, o, BH, N, D))
     return cuda_fail("cuTensorMapEncodeTiled (q/k/v/o)");
   fa::FwdParams p{};
   p.lse = lse;
+  p.o_hp = o_hp;
   if (st) {
     p.st_rm = st->rm;
     p.st_rs = st->rs;
@@ -210,11 +205,32 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   const int n_sm = sm_count();
   if (n_sm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)");
   const long long items = static_cast<long long>(p.n_qblk) * BH;
-  const long long slots = static_cast<long long>(n_sm) * L::CTAS_PER_SM;
-  const unsigned grid = static_cast<unsigned>(items < slots ? items : slots);
-  LaunchTimer tm(FA_KERNEL_FWD, stream);
-  cudaError_t e = launch_pdl(fa::fa_fwd_kernel<D>, dim3(grid), dim3(L::THREADS), L::SMEM_BYTES, stream, mq, mk, mv, mo, p);
-  tm.done();
+  auto launch = [&](auto kernel, int smem, int ctas_per_sm) {
+    const long long slots = static_cast<long long>(n_sm) * ctas_per_sm;
+    const unsigned grid = static_cast<unsigned>(items < slots ? items : slots);
+    LaunchTimer tm(FA_KERNEL_FWD, stream);
+    const cudaError_t err = launch_pdl(kernel, dim3(grid), dim3(384), smem, stream, mq, mk, mv, mo, p);
+    tm.done();
+    return err;
+  };
+  cudaError_t e;
+  if (o_hp == nullptr) {
+    using L = fa::FwdLayout<D, false>;
+    static bool attr = false;
+    if (!attr) {
+      if (!set_smem(fa::fa_fwd_kernel<D, false>, L::SMEM_BYTES)) return FA_ERR_CUDA;
+      attr = true;
+    }
+    e = launch(fa::fa_fwd_kernel<D, false>, L::SMEM_BYTES, L::CTAS_PER_SM);
+  } else {
+    using L = fa::FwdLayout<D, true>;
+    static bool attr = false;
+    if (!attr) {
+      if (!set_smem(fa::fa_fwd_kernel<D, true>, L::SMEM_BYTES)) return FA_ERR_CUDA;
+      attr = true;
+    }
+    e = launch(fa::fa_fwd_kernel<D, true>, L::SMEM_BYTES, L::CTAS_PER_SM);
+  }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : cuda_fail("fa_fwd_kernel launch", e);
 }
@@ -227,9 +243,9 @@ int grid_for(long long work, int per_block) {
 }
 
 template <int D>
-fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
-                     const float* row_m, void* dq, void* dk, void* dv, uint8_t* ws, int BH, int N, int causal,
-                     int mode, cudaStream_t stream) {
+fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, bool o_is_hp, const void* dO,
+                     const float* lse, const float* row_m, void* dq, void* dk, void* dv, uint8_t* ws, int BH, int N,
+                     int causal, int mode, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
   using LP = fa::BwdPipeLayout;
   static bool attr = false;
@@ -251,9 +267,13 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   {
     constexpr int rows_per_block = 8 * (32 / (D / 8)) * 4;  // 8 warps x rows per group x 4 groups
     LaunchTimer tm(FA_KERNEL_BWD_DELTA, stream);
-    cudaError_t e = launch_pdl(fa::fa_bwd_delta_kernel<D>, dim3(grid_for(rows, rows_per_block)), dim3(256), 0,
-                               stream, static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO),
-                               delta, dq_acc, rows);
+    const dim3 grid(grid_for(rows, rows_per_block));
+    cudaError_t e =
+        o_is_hp ? launch_pdl(fa::fa_bwd_delta_kernel<D, float>, grid, dim3(256), 0, stream,
+                             static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows)
+                : launch_pdl(fa::fa_bwd_delta_kernel<D, __nv_bfloat16>, grid, dim3(256), 0, stream,
+                             static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta,
+                             dq_acc, rows);
     tm.done();
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("fa_bwd_delta_kernel launch", e);
@@ -343,16 +363,24 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   return round256(rows * 4) + round256(rows * static_cast<size_t>(d) * 4);
 }
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const fa_row_stats* stats, int B,
-                 int H, int N, int d, int causal, int softmax_mode, float beta, void* stream) {
+}  // extern "C"
+
+namespace {
+
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* o_hp, bool want_hp, float* lse,
+                   const fa_row_stats* stats, int B, int H, int N, int d, int causal, int softmax_mode, float beta,
+                   void* stream) {
   if (!shape_ok(B, H, N, d)) return FA_ERR_INVALID_ARG;
-  if (softmax_mode != FA_SOFTMAX_STANDARD && softmax_mode != FA_SOFTMAX_STABILIZED) return FA_ERR_INVALID_ARG;
-  if (softmax_mode == FA_SOFTMAX_STABILIZED && !(std::isfinite(beta) && beta > 1.0f)) return FA_ERR_INVALID_ARG;
+  if (softmax_mode != FA_SOFTMAX_STANDARD && softmax_mode != FA_SOFTMAX_STABILIZED &&
+      softmax_mode != FA_SOFTMAX_STABILIZED_MARGIN)
+    return FA_ERR_INVALID_ARG;
+  if (softmax_mode != FA_SOFTMAX_STANDARD && !(std::isfinite(beta) && beta > 1.0f)) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
-  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+  if (!q || !k || !v || !o || !lse || (want_hp && !o_hp)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (want_hp && !aligned16(o_hp)))
     return FA_ERR_INVALID_ARG;
   if (stats) {
     const void* ptrs[4] = {stats->rm, stats->rs, stats->m, stats->pbar_max};
@@ -361,21 +389,24 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   }
   const int BH = B * H;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_fwd<64>(q, k, v, o, lse, stats, BH, N, causal, softmax_mode, beta, s);
-  return launch_fwd<128>(q, k, v, o, lse, stats, BH, N, causal, softmax_mode, beta, s);
+  if (d == 64) return launch_fwd<64>(q, k, v, o, o_hp, lse, stats, BH, N, causal, softmax_mode, beta, s);
+  return launch_fwd<128>(q, k, v, o, o_hp, lse, stats, BH, N, causal, softmax_mode, beta, s);
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
-                 const float* row_m, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
-                 int H, int N, int d, int causal, int softmax_mode, float beta, void* stream) {
+fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, bool o_is_hp, const void* dO,
+                   const float* lse, const float* row_m, void* dq, void* dk, void* dv, void* workspace,
+                   size_t workspace_bytes, int B, int H, int N, int d, int causal, int softmax_mode, float beta,
+                   void* stream) {
   if (!shape_ok(B, H, N, d)) return FA_ERR_INVALID_ARG;
-  if (softmax_mode != FA_SOFTMAX_STANDARD && softmax_mode != FA_SOFTMAX_STABILIZED) return FA_ERR_INVALID_ARG;
-  if (softmax_mode == FA_SOFTMAX_STABILIZED && !(std::isfinite(beta) && beta > 1.0f)) return FA_ERR_INVALID_ARG;
+  if (softmax_mode != FA_SOFTMAX_STANDARD && softmax_mode != FA_SOFTMAX_STABILIZED &&
+      softmax_mode != FA_SOFTMAX_STABILIZED_MARGIN)
+    return FA_ERR_INVALID_ARG;
+  if (softmax_mode != FA_SOFTMAX_STANDARD && !(std::isfinite(beta) && beta > 1.0f)) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
-  if (softmax_mode == FA_SOFTMAX_STABILIZED && !row_m) return FA_ERR_INVALID_ARG;
+  if (softmax_mode != FA_SOFTMAX_STANDARD && !row_m) return FA_ERR_INVALID_ARG;
   const void* a16[8] = {q, k, v, o, dO, dq, dk, dv};
   for (const void* pp : a16)
     if (!aligned16(pp)) return FA_ERR_INVALID_ARG;
@@ -387,8 +418,41 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   const int BH = B * H;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (d == 64) return launch_bwd<64>(q, k, v, o, dO, lse, row_m, dq, dk, dv, ws, BH, N, causal, softmax_mode, s);
-  return launch_bwd<128>(q, k, v, o, dO, lse, row_m, dq, dk, dv, ws, BH, N, causal, softmax_mode, s);
+  // both stabilised modes recompute P the same way (P = exp(S - m) / l)
+  const int bwd_mode = softmax_mode == FA_SOFTMAX_STANDARD ? 0 : 1;
+  if (d == 64)
+    return launch_bwd<64>(q, k, v, o, o_is_hp, dO, lse, row_m, dq, dk, dv, ws, BH, N, causal, bwd_mode, s);
+  return launch_bwd<128>(q, k, v, o, o_is_hp, dO, lse, row_m, dq, dk, dv, ws, BH, N, causal, bwd_mode, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const fa_row_stats* stats, int B,
+                 int H, int N, int d, int causal, int softmax_mode, float beta, void* stream) {
+  return fwd_impl(q, k, v, o, nullptr, false, lse, stats, B, H, N, d, causal, softmax_mode, beta, stream);
+}
+
+fa_status fa_fwd_o_hp(const void* q, const void* k, const void* v, void* o, float* o_hp, float* lse,
+                      const fa_row_stats* stats, int B, int H, int N, int d, int causal, int softmax_mode, float beta,
+                      void* stream) {
+  return fwd_impl(q, k, v, o, o_hp, true, lse, stats, B, H, N, d, causal, softmax_mode, beta, stream);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 const float* row_m, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
+                 int H, int N, int d, int causal, int softmax_mode, float beta, void* stream) {
+  return bwd_impl(q, k, v, o, false, dO, lse, row_m, dq, dk, dv, workspace, workspace_bytes, B, H, N, d, causal,
+                  softmax_mode, beta, stream);
+}
+
+fa_status fa_bwd_o_hp(const void* q, const void* k, const void* v, const float* o_hp, const void* dO,
+                      const float* lse, const float* row_m, void* dq, void* dk, void* dv, void* workspace,
+                      size_t workspace_bytes, int B, int H, int N, int d, int causal, int softmax_mode, float beta,
+                      void* stream) {
+  return bwd_impl(q, k, v, o_hp, true, dO, lse, row_m, dq, dk, dv, workspace, workspace_bytes, B, H, N, d, causal,
+                  softmax_mode, beta, stream);
 }
 
 const char* fa_last_error_string(void) { return g_last_error; }

@@ -19,13 +19,22 @@
  *                                               P_bar; the rm > 0 rule with
  *                                               |rm| replaced by 1 is used
  *           rm       otherwise
+ *   m2    = m + margin rule                        (FA_SOFTMAX_STABILIZED_MARGIN)
+ *           on rows with rs > 1 where m - rm < 2^-8 (fp32 subtraction),
+ *           m2 = rm + 2^-8 (fp32 add); otherwise m2 = m.  The rule above keeps
+ *           the fp32 max(P_bar) below 1, but bf16(P_bar) still rounds to 1
+ *           when m - rm < 2^-9; with the margin, exp(rm - m2) <= exp(-2^-8)
+ *           and its bf16 value is below 1 too.  (The pages give the fp32
+ *           rule; the margin carries their goal, max(P_bar) < 1, to the bf16
+ *           operand of the P V product.)
  *   P_bar = exp(S - m),  l = rowsum(P_bar),  P = P_bar / l,  O = P V
  *   lse   = m + ln(l)                          (natural logarithm)
  *
  *   backward: delta = rowsum(dO o O), dV = P^T dO, dP = dO V^T,
  *             dS = P o (dP - delta), dQ = dS K * scale, dK = dS^T Q * scale,
  *   with P recomputed as exp(S - lse) (standard) or as
- *   exp(S - m) * (1/l), l = exp(lse - m) (stabilised, m from the forward).
+ *   exp(S - m) * (1/l), l = exp(lse - m) (both stabilised modes, m from the
+ *   forward).
  *
  * Layout: Q, K, V, O, dO, dQ, dK, dV are bf16 arrays [B, H, N, d], contiguous
  * (d fastest), base addresses 16-byte aligned.  lse, delta and the row
@@ -47,7 +56,7 @@
  * Domain: d in {64, 128}; any N >= 0 (a ragged last tile of fewer than 128
  * rows is masked); B, H >= 0, and a problem with B*H*N == 0 is a valid
  * no-op; B*H*N*d < 2^40 and B*H*ceil(N/128) < 2^31.  beta must be finite
- * and > 1 in stabilised mode (ignored in standard mode).
+ * and > 1 in the stabilised modes (ignored in standard mode).
  */
 #ifndef FA_B200_H_
 #define FA_B200_H_
@@ -68,7 +77,11 @@ typedef enum {
   FA_ERR_TIMEOUT = 5       /* a kernel gave up on a bounded wait (see fa_device_error) */
 } fa_status;
 
-typedef enum { FA_SOFTMAX_STANDARD = 0, FA_SOFTMAX_STABILIZED = 1 } fa_softmax_mode;
+typedef enum {
+  FA_SOFTMAX_STANDARD = 0,
+  FA_SOFTMAX_STABILIZED = 1,
+  FA_SOFTMAX_STABILIZED_MARGIN = 2
+} fa_softmax_mode;
 
 /* Optional per-row outputs of the forward, each [B, H, N]; any may be NULL.
  * rm: row max of S; rs: its tie count; m: the shift used (this is what
@@ -95,8 +108,8 @@ size_t fa_bwd_workspace_delta_offset(int B, int H, int N, int d);
 size_t fa_bwd_workspace_dq_offset(int B, int H, int N, int d);
 
 /* Backward.  Inputs q, k, v, o, dO (bf16), lse (fp32, from fa_fwd), row_m
- * (fp32 shift m from fa_fwd's stats; required in stabilised mode, ignored
- * otherwise); outputs dq, dk, dv (bf16).  workspace: caller-owned device
+ * (fp32 shift m from fa_fwd's stats; required in the stabilised modes,
+ * ignored otherwise); outputs dq, dk, dv (bf16).  workspace: caller-owned device
  * memory of at least fa_bwd_workspace_bytes, 256-byte aligned; its contents
  * on entry do not matter and on exit hold delta and the fp32 dQ.  Launches
  * three kernels on `stream`: delta, main (dK, dV, partial dQ), dQ convert.
@@ -104,6 +117,28 @@ size_t fa_bwd_workspace_dq_offset(int B, int H, int N, int d);
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  const float* row_m, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
                  int H, int N, int d, int causal, int softmax_mode, float beta, void* stream);
+
+/* High-precision O (the pages' O_hp; reading of their localisation remedy:
+ * keep the rounded O_lp out of the delta term of the backward).
+ *
+ * fa_fwd_o_hp: as fa_fwd (the bf16 o and every other output are the same,
+ * bit for bit), and also writes o_hp, fp32 [B, H, N, d] (16-byte aligned,
+ * caller-owned): O with P_bar carried to about 16 bits -- P_bar is split into
+ * P_hi = bf16(P_bar) and P_lo = bf16(P_bar - P_hi), the two parts are
+ * multiplied by V into separate fp32 accumulators and o_hp = (O_hi + O_lo)/l.
+ * The bf16 o is O_hi / l rounded, as in fa_fwd.  Costs a second P V product
+ * and a 512-column TMEM allocation (one CTA per SM).
+ *
+ * fa_bwd_o_hp: as fa_bwd, with delta = rowsum(dO o O_hp) taken from the fp32
+ * O instead of the bf16 one; every other step is fa_bwd's.  Same workspace,
+ * same errors (o_hp NULL or misaligned: FA_ERR_INVALID_ARG). */
+fa_status fa_fwd_o_hp(const void* q, const void* k, const void* v, void* o, float* o_hp, float* lse,
+                      const fa_row_stats* stats, int B, int H, int N, int d, int causal, int softmax_mode, float beta,
+                      void* stream);
+fa_status fa_bwd_o_hp(const void* q, const void* k, const void* v, const float* o_hp, const void* dO,
+                      const float* lse, const float* row_m, void* dq, void* dk, void* dv, void* workspace,
+                      size_t workspace_bytes, int B, int H, int N, int d, int causal, int softmax_mode, float beta,
+                      void* stream);
 
 /* Static description of a status code. */
 const char* fa_status_string(fa_status s);

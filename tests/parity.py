@@ -52,6 +52,30 @@ def run_gpu(w, mode: int, beta: float = 2.0, dev="cuda:0", bwd: bool = True):
     return {k_: v_.float().cpu().numpy() if v_.dtype != torch.int32 else v_.cpu().numpy() for k_, v_ in out.items()}
 
 
+def run_gpu_o_hp(w, mode: int, beta: float = 2.0, dev="cuda:0"):
+    """Forward with the fp32 O (fa_fwd_o_hp), backward with delta from it
+    (fa_bwd_o_hp)."""
+    q, k, v, do = (to_dev(x, dev) for x in (w.q, w.k, w.v, w.do))
+    B, H, N, d = q.shape
+    o = torch.empty_like(q)
+    o_hp = torch.empty(B, H, N, d, device=dev, dtype=torch.float32)
+    lse = torch.empty(B, H, N, device=dev, dtype=torch.float32)
+    st = fa.RowStats.empty(B, H, N, dev)
+    fa.fa_fwd_o_hp(q, k, v, o, o_hp, lse, st, w.causal, mode, beta)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), device=dev, dtype=torch.uint8)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    fa.fa_bwd_o_hp(q, k, v, o_hp, do, lse, st.m, dq, dk, dv, ws, w.causal, mode, beta)
+    off_delta, _ = fa.fa_bwd_workspace_offsets(B, H, N, d)
+    delta = ws[off_delta:off_delta + B * H * N * 4].view(torch.float32).view(B, H, N)
+    out = {"o": o, "o_hp": o_hp, "lse": lse, "m": st.m, "dq": dq, "dk": dk, "dv": dv, "delta": delta}
+    torch.cuda.synchronize(dev)
+    status, word = fa.fa_device_error()
+    assert status == 0, f"device error word {word:#x}"
+    res = {k_: v_.float().cpu().numpy() for k_, v_ in out.items()}
+    res["o_bits"] = o.view(torch.int16).cpu().numpy()
+    return res
+
+
 def head_slice(x, pairs):
     return np.stack([x[b, h] for b, h in pairs])[None]
 

@@ -70,7 +70,9 @@ def test_fwd_argument_errors(lib):
     assert fwd(lib, beta=0.5) == _abi.FA_ERR_INVALID_ARG
     assert fwd(lib, beta=float("nan")) == _abi.FA_ERR_INVALID_ARG
     assert fwd(lib, beta=float("inf")) == _abi.FA_ERR_INVALID_ARG
-    assert fwd(lib, mode=2) == _abi.FA_ERR_INVALID_ARG
+    assert fwd(lib, mode=3) == _abi.FA_ERR_INVALID_ARG
+    assert fwd(lib, mode=-1) == _abi.FA_ERR_INVALID_ARG
+    assert fwd(lib, mode=2, beta=1.0) == _abi.FA_ERR_INVALID_ARG  # the margin mode is a stabilised mode
     assert fwd(lib, causal=2) == _abi.FA_ERR_INVALID_ARG
     assert fwd(lib, B=-1) == _abi.FA_ERR_INVALID_ARG
     assert fwd(lib, q=NUL) == _abi.FA_ERR_INVALID_ARG
@@ -97,9 +99,30 @@ def test_bwd_argument_errors(lib):
     assert bwd(lib, ws=ctypes.c_void_p(0x100010)) == _abi.FA_ERR_WORKSPACE  # not 256-byte aligned
     assert bwd(lib, ws=None) == _abi.FA_ERR_WORKSPACE
     assert bwd(lib, row_m=None) == _abi.FA_ERR_INVALID_ARG                 # required when stabilised
+    assert bwd(lib, row_m=None, mode=2) == _abi.FA_ERR_INVALID_ARG
+    assert bwd(lib, mode=3) == _abi.FA_ERR_INVALID_ARG
     assert bwd(lib, q=MIS) == _abi.FA_ERR_INVALID_ARG
     assert bwd(lib, d=80) == _abi.FA_ERR_UNSUPPORTED
     assert bwd(lib, beta=1.0) == _abi.FA_ERR_INVALID_ARG
+
+
+def test_o_hp_entry_points_argument_errors(lib):
+    # forward: o_hp is required and 16-byte aligned; everything else as fa_fwd
+    def fwd_hp(o_hp=P, mode=1, N=128, d=64):
+        return lib.fa_fwd_o_hp(P, P, P, P, o_hp, P, None, 1, 2, N, d, 1, mode, 2.0, None)
+    assert fwd_hp(o_hp=NUL) == _abi.FA_ERR_INVALID_ARG
+    assert fwd_hp(o_hp=MIS) == _abi.FA_ERR_INVALID_ARG
+    assert fwd_hp(mode=3) == _abi.FA_ERR_INVALID_ARG
+    assert fwd_hp(d=96) == _abi.FA_ERR_UNSUPPORTED
+    assert fwd_hp(N=0, o_hp=NUL) == _abi.FA_OK  # empty problem: nothing to write
+    # backward: same checks as fa_bwd with the fp32 O in place of the bf16 one
+    def bwd_hp(o_hp=P, ws_bytes=1 << 30, row_m=P, mode=1):
+        return lib.fa_bwd_o_hp(P, P, P, o_hp, P, P, row_m, P, P, P, ctypes.c_void_p(0x100000), ws_bytes, 1, 2, 128,
+                               64, 1, mode, 2.0, None)
+    assert bwd_hp(o_hp=NUL) == _abi.FA_ERR_INVALID_ARG
+    assert bwd_hp(o_hp=MIS) == _abi.FA_ERR_INVALID_ARG
+    assert bwd_hp(row_m=None) == _abi.FA_ERR_INVALID_ARG
+    assert bwd_hp(ws_bytes=16) == _abi.FA_ERR_WORKSPACE
 
 
 def test_workspace_layout(lib):

@@ -10,6 +10,7 @@ import pytest
 import torch
 
 import workloads
+from oracle import bf16
 from tests import parity as P
 
 pytestmark = pytest.mark.gpu
@@ -21,14 +22,16 @@ def _small(name, B, H, N, seed=None):
 
 def _check_fix_invariants(gpu, mode):
     tied = gpu["rs"] > 1
-    if mode == 1:
+    if mode in (1, 2):
         assert np.all(gpu["pbar_max"][tied] < 1.0)
         assert np.all(gpu["pbar_max"][~tied] == 1.0)
     else:
         assert np.all(gpu["pbar_max"] == 1.0)
+    if mode == 2:  # the margin keeps the bf16 operand below 1 as well
+        assert np.all(bf16.round_bf16(gpu["pbar_max"][tied].astype(np.float32)) < 1.0)
 
 
-@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("mode", [0, 1, 2])
 def test_tiny_exact_stats(cuda_device, mode):
     w = workloads.make("tiny")
     gpu = P.run_gpu(w, mode)
@@ -49,7 +52,7 @@ def _d128_case(N, causal, tie_scale):
     return w
 
 
-@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("mode", [0, 1, 2])
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("N", [384, 200])
@@ -100,7 +103,7 @@ def test_two_hot_ties_within_bf16_floor(cuda_device, causal, N):
         P.assert_close(key, gpu[key], ref[key])
 
 
-@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("mode", [0, 1, 2])
 def test_tiestress_small_exact(cuda_device, mode):
     """Quantised scores (exact in fp32): rm, rs, m bit-exact, all three tie classes."""
     w = workloads.make("tiestress", B=1, H=2, N=640)
@@ -110,8 +113,54 @@ def test_tiestress_small_exact(cuda_device, mode):
     _check_fix_invariants(gpu, mode)
     cls = w.notes["tie_class"]
     assert np.all(gpu["rs"][cls >= 0] == 2)
-    if mode == 1:
-        assert np.all(gpu["m"][cls == 2] == 1.0) and np.all(gpu["m"][cls == 1] == 0.0)
+    if mode in (1, 2):
+        assert np.all(gpu["m"][cls == 2] == 1.0)
+        if mode == 1:
+            assert np.all(gpu["m"][cls == 1] == 0.0)
+
+
+def _margin_case(N, causal):
+    """Every row has a tied maximum rm = 2^-9 (1/8-grid inputs, exact scores):
+    q = +-e_i / 8 on dims 0-3; keys 0 and N/2 are +(1/8) there, the rest -(1/8)."""
+    rng = np.random.default_rng(N)
+    q = np.zeros((1, 2, N, 64), np.float32)
+    k = np.zeros((1, 2, N, 64), np.float32)
+    for i in range(N):
+        q[:, :, i, i % 4] = 0.125 if i % 2 == 0 else -0.125
+    k[:, :, :, :4] = -0.125
+    k[:, :, 0, :4] = 0.125
+    k[:, :, N // 2, :4] = 0.125
+    mk = lambda: workloads.to_bf16_values(rng.standard_normal((1, 2, N, 64)).astype(np.float32))
+    return workloads.Workload("margin", 1, 2, N, 64, causal, 0, q, k, mk(), mk(), np.zeros((1, 2, N), bool))
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_margin_mode_small_ties(cuda_device, causal):
+    """Tied maxima of size 2^-9: the fp32 rule leaves bf16(P_bar) = 1 on those
+    rows; the margin mode moves m by 2^-8 (bit-exact against the oracle) and
+    keeps it below 1.  Forward outputs and dV are compared with the oracle;
+    dQ and dK of this construction are sums of nearly uniform dS over two
+    key (query) values, pure cancellation below the bf16 dS rounding, so
+    their parity is left to the general grid (which runs mode 2 too)."""
+    w = _margin_case(384, causal)
+    for mode in (1, 2):
+        gpu = P.run_gpu(w, mode)
+        ref = P.oracle(w, mode, o_gpu=gpu["o"])
+        P.assert_close("o", gpu["o"], ref["o"])
+        P.assert_close("dv", gpu["dv"], ref["dv"])
+        assert np.abs(gpu["lse"] - ref["lse"]).max() <= P.LSE_ABS
+        for key in ("rm", "rs", "m"):
+            assert np.array_equal(gpu[key], ref[key]), key
+        _check_fix_invariants(gpu, mode)
+        tied = gpu["rs"] > 1
+        small = tied & (np.abs(gpu["rm"]) < 2.0 ** -8)
+        assert small.sum() > 100
+        b = bf16.round_bf16(gpu["pbar_max"][small].astype(np.float32))
+        if mode == 1:
+            assert np.all(b == 1.0)
+        else:
+            assert np.all(b < 1.0)
+            assert np.all(gpu["m"][small] == gpu["rm"][small] + np.float32(2.0 ** -8))
 
 
 def test_empty_problem_is_noop(cuda_device):
@@ -191,3 +240,72 @@ def test_modes_agree_on_gpu(cuda_device):
     g1 = P.run_gpu(w, 1)
     for key in ("o", "dq", "dk", "dv"):
         P.assert_close(key, g1[key], g0[key])
+
+
+# --------------------------------------- high-precision O for the delta term
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_o_hp_forward(cuda_device, d):
+    """fa_fwd_o_hp: o_hp carries P_bar to ~16 bits, so it matches the float64
+    O far inside the bf16 tolerance (1e-4 of max|O| here, against 1e-2 for
+    the bf16 o); every other output equals fa_fwd's bit for bit."""
+    w = workloads.make("g2s", B=1, H=2, N=200, seed=7) if d == 64 else _d128_case(200, True, 0.25)
+    hp = P.run_gpu_o_hp(w, 1)
+    lp = P.run_gpu(w, 1)
+    ref = P.oracle(w, 1, o_gpu=hp["o"])
+    err_hp = np.abs(hp["o_hp"] - ref["o"]).max() / np.abs(ref["o"]).max()
+    err_lp = np.abs(lp["o"] - ref["o"]).max() / np.abs(ref["o"]).max()
+    print(f"d={d}: max |O - O_float64| / max|O|: o_hp {err_hp:.2e}, bf16 o {err_lp:.2e}")
+    assert err_hp <= 1e-4
+    for key in ("o", "lse", "m"):
+        assert np.array_equal(lp[key], hp[key]), key
+
+
+@pytest.mark.parametrize("name", ["tiestress", "g2s"])
+def test_o_hp_backward_removes_the_delta_bias(cuda_device, name):
+    """The pages' remedy (P in higher precision wherever it feeds dP): delta
+    from the ~16-bit-P O_hp is the float64 delta to ~1e-5, and the gradients
+    come close to the chained float64 gradient; with delta from the bf16 O
+    they carry its error (biased on rows with tied maxima)."""
+    w = workloads.make(name).heads([(0, 0)])
+    lp = P.run_gpu(w, 1)
+    hp = P.run_gpu_o_hp(w, 1)
+    ref = P.oracle(w, 1)   # chained: delta from the oracle's float64 O
+    scale = np.abs(ref["delta"]).max()
+    d_lp = np.abs(lp["delta"] - ref["delta"]).max() / scale
+    d_hp = np.abs(hp["delta"] - ref["delta"]).max() / scale
+    print(f"{name}: max |delta - delta(float64 O)| / max|delta|: bf16 O {d_lp:.2e}, O_hp {d_hp:.2e}")
+    assert d_hp <= 1e-4 and d_hp < d_lp
+    for key in ("dq", "dk", "dv"):
+        e_lp = np.abs(lp[key] - ref[key]).max() / np.abs(ref[key]).max()
+        e_hp = np.abs(hp[key] - ref[key]).max() / np.abs(ref[key]).max()
+        print(f"{name} {key}: max err vs chained float64: delta from bf16 O {e_lp:.4f}, from O_hp {e_hp:.4f}")
+        P.assert_close(key, hp[key], ref[key])
+
+
+# ---------------------------------------------- bias diagnostic (negative V)
+
+@pytest.mark.parametrize("name", ["tiestress", "tiny"])
+def test_bias_diagnostic_negative_v(cuda_device, name):
+    """The pages' Figure 6 question on this hardware: on rows with a tied
+    maximum, does O drift in one direction on the value columns whose mean is
+    negative?  Reports mean(O_gpu - O_float64) over the tied rows, for the
+    negative-mean columns and for the rest, and the mean delta error, in all
+    three modes.  Here the P V product accumulates in fp32 (TMEM) and only
+    P_bar and O are rounded to bf16 (RNE); the bound is one bf16 step of the
+    mean |O| (2^-8 relative), a drift of that size would be visible in every
+    row."""
+    w = workloads.make(name) if name == "tiny" else workloads.make(name).heads([(0, 0)])
+    neg_cols = 16 if name == "tiny" else 32
+    for mode in (0, 1, 2):
+        gpu = P.run_gpu(w, mode)
+        ref = P.oracle(w, mode)
+        tied = ref["rs"] > 1
+        err = gpu["o"] - ref["o"]
+        e_neg = err[tied][:, :neg_cols].mean()
+        e_rest = err[tied][:, neg_cols:].mean()
+        scale = np.abs(ref["o"][tied]).mean()
+        d_err = (gpu["delta"] - ref["delta"])[tied].mean()
+        print(f"{name} mode {mode}: tied rows {int(tied.sum())}, mean O error on negative-mean columns "
+              f"{e_neg:+.3e}, other columns {e_rest:+.3e} (mean |O| {scale:.3f}); mean delta error {d_err:+.3e}")
+        assert abs(e_neg) <= 2.0 ** -8 * scale and abs(e_rest) <= 2.0 ** -8 * scale
