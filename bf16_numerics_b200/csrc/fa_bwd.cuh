@@ -43,22 +43,52 @@ namespace fa {
 // lanes per row (8 elements of dO per lane); every warp takes U row groups at
 // a time and issues all of their loads before using any, so enough bytes are
 // in flight to cover the DRAM latency.
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
-  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
-  const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+// 8 consecutive elements of O as they sit in memory (16 bytes of bf16 or
+// 32 bytes of fp32), and their dot product with 8 bf16 elements of dO
+template <typename OT>
+struct ORaw;
+template <>
+struct ORaw<__nv_bfloat16> {
+  uint4 v;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { v = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void zero() { v = make_uint4(0u, 0u, 0u, 0u); }
+  __device__ __forceinline__ float dot(const uint4& d, float acc) const {
+    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&v);
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&d);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 x = __bfloat1622float2(pa[i]);
-    f[2 * i] = x.x;
-    f[2 * i + 1] = x.y;
+    for (int i = 0; i < 4; ++i) {
+      const float2 a = __bfloat1622float2(pa[i]), b = __bfloat1622float2(pb[i]);
+      acc = fmaf(a.x, b.x, acc);
+      acc = fmaf(a.y, b.y, acc);
+    }
+    return acc;
   }
-}
-__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
+};
+template <>
+struct ORaw<float> {
+  float4 lo, hi;
+  __device__ __forceinline__ void load(const float* p) {
+    lo = __ldg(reinterpret_cast<const float4*>(p));
+    hi = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ __forceinline__ void zero() { lo = hi = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ float dot(const uint4& d, float acc) const {
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&d);
+    float2 b = __bfloat1622float2(pb[0]);
+    acc = fmaf(lo.x, b.x, acc);
+    acc = fmaf(lo.y, b.y, acc);
+    b = __bfloat1622float2(pb[1]);
+    acc = fmaf(lo.z, b.x, acc);
+    acc = fmaf(lo.w, b.y, acc);
+    b = __bfloat1622float2(pb[2]);
+    acc = fmaf(hi.x, b.x, acc);
+    acc = fmaf(hi.y, b.y, acc);
+    b = __bfloat1622float2(pb[3]);
+    acc = fmaf(hi.z, b.x, acc);
+    acc = fmaf(hi.w, b.y, acc);
+    return acc;
+  }
+};
 
 template <int D, typename OT>
 __global__ void __launch_bounds__(256)
@@ -74,16 +104,17 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
   grid_launch_dependents();
   grid_dependency_wait();  // O comes from the forward grid
   for (long long r0 = warp_global * (RPW * U); r0 < rows; r0 += n_warps * (RPW * U)) {
-    float a[U][8], b[U][8];
+    ORaw<OT> a[U];
+    uint4 b[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const long long r = r0 + u * RPW + sub;
       if (r < rows) {
-        load8(o + r * D + 8 * li, a[u]);
-        load8(dO + r * D + 8 * li, b[u]);
+        a[u].load(o + r * D + 8 * li);
+        b[u] = __ldg(reinterpret_cast<const uint4*>(dO + r * D) + li);
       } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a[u][i] = b[u][i] = 0.f;
+        a[u].zero();
+        b[u] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
 #pragma unroll
@@ -97,9 +128,7 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc = fmaf(a[u][i], b[u][i], acc);
+      float acc = a[u].dot(b[u], 0.f);
 #pragma unroll
       for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
       const long long r = r0 + u * RPW + sub;

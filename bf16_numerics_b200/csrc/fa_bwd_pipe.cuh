@@ -225,8 +225,10 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       bool ok = true;
       for (; ok && cur.valid; cur.next_item()) {
         // the item's first query blocks go ahead of its K/V, which must wait
-        // for the previous item's products to release the K/V buffers
-        const int first = cur.n < 2 ? cur.n : 2;
+        // for the previous item's products to release the K/V buffers; at the
+        // cold start only block 0 goes first, and the rest of the ring waits
+        // until the first products' operands (K, V, Q_0, dO_0) have arrived
+        const int first = cur.r == 0 ? 1 : (cur.n < 2 ? cur.n : 2);
         for (int i = 0; ok && i < first; ++i) ok = load_q(i, g + i);
         if (!ok) break;
         if (cur.r > 0 && !wait(bar(L::KV_EMPTY), (cur.r - 1) & 1, 1)) break;
@@ -234,6 +236,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         tma_load_3d(base + L::K_OFF, &tm_k, bar(L::KV_FULL), 0, cur.kblk * L::B, cur.bh);
         tma_load_3d(base + L::V_OFF, &tm_v, bar(L::KV_FULL), 0, cur.kblk * L::B, cur.bh);
         last_r = cur.r;
+        if (cur.r == 0 && (!wait(bar(L::KV_FULL), 0, 23) || !wait(bar(L::Q_FULL), 0, 24))) break;
         for (int i = first; ok && i < cur.n; ++i) ok = load_q(i, g + i);
         g += cur.n;
       }

@@ -252,6 +252,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tma_load_3d(base + L::K_OFF + s * L::TILE + hh * L::HALF, &tm_k, bar(L::K_FULL + s), 64 * hh,
                         j * L::BN, cur.bh);
           k_issued = gt + 1;
+          if (gt == 0) {
+            // cold start: let the first Q K^T's operands arrive before the
+            // rest of the rings competes with them for DRAM
+            if (!wait(bar(L::Q_FULL), 0, 23) || !wait(bar(L::K_FULL), 0, 24)) { ok = false; break; }
+          }
           if (u > 0 && !wait(bar(L::V_EMPTY + s), (u - 1) & 1, 3)) { ok = false; break; }
           mbar_expect_tx(bar(L::V_FULL + s), L::TILE);
           for (int hh = 0; hh < D / 64; ++hh)
