@@ -322,6 +322,39 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+
+// 2^y for a pair of fp32 arguments on the FMA and integer pipes instead of
+// the MUFU (which the exponentials of the softmax keep busy).  Cody-Waite
+// range reduction (Cody & Waite, "Software Manual for the Elementary
+// Functions", 1980): y = k + r with k = round(y) taken by adding and removing
+// 1.5 * 2^23, r in [-1/2, 1/2] exact; 2^r by a degree-5 polynomial with
+// constant term 1, fitted for this library by relative least squares with
+// Lawson reweighting on [-1/2, 1/2] (max relative error 1.9e-7 in fp32
+// Horner form, the accuracy class of ex2.approx); 2^k by adding k to the
+// exponent field.  y = 0 gives exactly 1.  Arguments below -126 (masked
+// scores are -inf) are clamped to -126: the result is then 2^-126 instead of
+// 0, far below anything that reaches a bf16 operand or the fp32 row sum.
+__device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t y) {
+  float y0, y1;
+  f2_unpack(y, y0, y1);
+  const uint64_t yc = f2_pack(fmaxf(y0, -126.f), fmaxf(y1, -126.f));
+  const uint64_t kMagic = f2_pack(12582912.f, 12582912.f);  // 1.5 * 2^23
+  const uint64_t t = f2_add(yc, kMagic);                     // 1.5 * 2^23 + k
+  const uint64_t r = f2_sub(yc, f2_sub(t, kMagic));          // y - k
+  uint64_t q = f2_fma(f2_pack(0.0013264636509120464f, 0.0013264636509120464f), r,
+                      f2_pack(0.009671482257544994f, 0.009671482257544994f));
+  q = f2_fma(q, r, f2_pack(0.05550733581185341f, 0.05550733581185341f));
+  q = f2_fma(q, r, f2_pack(0.24022242426872253f, 0.24022242426872253f));
+  q = f2_fma(q, r, f2_pack(0.6931470036506653f, 0.6931470036506653f));
+  q = f2_fma(q, r, f2_pack(1.f, 1.f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  // the low bits of t hold k (two's complement): shifting them to the
+  // exponent field drops the 1.5 * 2^23 part
+  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+}
 }  // namespace fa
 
 namespace fa {
