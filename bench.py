@@ -7,6 +7,10 @@ HBM.  The inputs (50 MB) fit in the 126 MB L2, so L2 is flushed (a 256 MiB
 write) before every timed step; the flush is outside the CUDA-event intervals.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload g2s|g2m|long|tiestress|tiny] [--mode 0|1|2]
+
+The default workload (GPT-2-small attention, g2s) is the headline; the other
+named workloads are the parity-test shapes and are timed the same way.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own copy of the
 workload (independent (batch, head) problems, no collective on the data path:
@@ -46,7 +50,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--mode", type=int, default=1, help="0 standard shift, 1 stabilised shift")
+    ap.add_argument("--mode", type=int, default=1, help="0 standard shift, 1 stabilised shift, 2 with margin")
+    ap.add_argument("--workload", default=WORKLOAD, help="workload name (workloads.CONFIGS)")
     ap.add_argument("--beta", type=float, default=2.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -168,12 +173,12 @@ def cpu_oracle_sample(w, mode, beta, seconds):
 
 
 # ------------------------------------------------------------------ ranks
-def rank_seed(rank: int) -> int:
+def rank_seed(rank: int, workload: str = WORKLOAD) -> int:
     """Seed of a rank's copy of the workload: same shapes on every rank (weak
     scaling), independent values."""
     import workloads
 
-    return workloads.CONFIGS[WORKLOAD][5] + rank
+    return workloads.CONFIGS[workload][5] + rank
 
 
 def rank_max(x: float, world: int, device=None) -> float:
@@ -193,13 +198,26 @@ def aggregate_tflops(world: int, flops_per_rank_step: float, steps: int, max_ms:
     return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
 
 
+WORKLOAD_TEXT = {
+    "g2s": ("GPT-2 small attention", "seeded synthetic N(0,1) Q,K,V,dO; key 0 duplicated, 10% of rows tied on it; "
+                                     "V cols 0-7 mean -0.75"),
+    "g2m": ("GPT-2 medium attention", "seeded synthetic Q,K ~ N(0,1.5^2), V,dO ~ N(0,1)"),
+    "long": ("long-context attention", "seeded synthetic N(0,1); key 0 duplicated, 5% of rows tied on it"),
+    "tiestress": ("tie-stress attention", "Q,K on the 1/8 grid, 25% of rows tied (rm > 0, < 0, == 0); "
+                                          "V, dO dims 0-31 mean -0.5"),
+    "tiny": ("tiny attention", "Q,K on the 1/8 grid; V cols 0-15 mean -1"),
+}
+MODE_TEXT = {0: "standard", 1: "stabilized", 2: "stabilized_margin"}
+
+
 def workload_config(w, mode, beta):
-    return {"workload": f"{w.name}: GPT-2 small attention B{w.B} H{w.H} N{w.N} d{w.d} causal, "
-                        f"{'stabilised' if mode == 1 else 'standard'} shift (beta={beta})",
+    what, inputs = WORKLOAD_TEXT.get(w.name, (w.name, "seeded synthetic"))
+    return {"workload": f"{w.name}: {what} B{w.B} H{w.H} N{w.N} d{w.d} {'causal' if w.causal else 'non-causal'}, "
+                        f"{MODE_TEXT[mode]} shift (beta={beta})",
             "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-            "softmax_mode": "stabilized" if mode == 1 else "standard", "beta": beta,
+            "softmax_mode": MODE_TEXT[mode], "beta": beta,
             "l2": "flushed before every timed step (256 MiB write, then a 256 MiB read of another buffer; outside the timed intervals)",
-            "inputs": "seeded synthetic N(0,1) Q,K,V,dO; key 0 duplicated, 10% of rows tied on it; V cols 0-7 mean -0.75"}
+            "inputs": inputs}
 
 
 def run_reference(args, rank, world):
@@ -207,7 +225,7 @@ def run_reference(args, rank, world):
 
     if rank != 0:
         return 0
-    w = workloads.make(WORKLOAD)
+    w = workloads.make(args.workload)
     per_step = min(1.0, 120.0 / max(1, args.steps + args.warmup))  # whole run bounded to ~2 min (>= 1 head/step)
     for _ in range(args.warmup):
         cpu_oracle_sample(w, args.mode, args.beta, per_step)
@@ -242,7 +260,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = workloads.make(WORKLOAD, seed=rank_seed(rank))
+    w = workloads.make(args.workload, seed=rank_seed(rank, args.workload))
     B, H, N, d = w.B, w.H, w.N, w.d
     mode, beta, causal = args.mode, args.beta, w.causal
 
