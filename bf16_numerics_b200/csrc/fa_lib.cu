@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -23,9 +24,8 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
@@ -33,7 +33,7 @@ EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
     else
       cudaGetLastError();
-  }
+  });
   return fn;
 }
 
@@ -88,11 +88,14 @@ struct TimingRec {
   int kernel;
   cudaEvent_t start, stop;
 };
-bool g_timing = false;
+// The timing records are shared by all host threads (one lock; timing is a
+// measurement aid and off by default).
+std::atomic<bool> g_timing{false};
+std::mutex g_timing_mutex;
 std::vector<TimingRec> g_recs;
 std::vector<cudaEvent_t> g_event_pool;
 
-cudaEvent_t take_event() {
+cudaEvent_t take_event() {  // caller holds g_timing_mutex
   if (!g_event_pool.empty()) {
     cudaEvent_t e = g_event_pool.back();
     g_event_pool.pop_back();
@@ -109,12 +112,14 @@ struct LaunchTimer {
   cudaEvent_t start = nullptr;
   LaunchTimer(int k, cudaStream_t s) : kernel(k), stream(s) {
     if (g_timing) {
+      std::lock_guard<std::mutex> lock(g_timing_mutex);
       start = take_event();
       if (start) cudaEventRecord(start, stream);
     }
   }
   void done() {
     if (g_timing && start) {
+      std::lock_guard<std::mutex> lock(g_timing_mutex);
       cudaEvent_t stop = take_event();
       if (stop) {
         cudaEventRecord(stop, stream);
@@ -156,9 +161,22 @@ bool set_smem(K kernel, int bytes) {
   return true;
 }
 
+// The dynamic shared memory limit of a kernel, raised once per device (the
+// attribute belongs to the kernel as loaded on the current device).
+template <typename K>
+bool ensure_smem(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return set_smem(kernel, bytes);
+  const uint64_t bit = uint64_t{1} << dev;
+  if (done_mask.load() & bit) return true;
+  if (!set_smem(kernel, bytes)) return false;
+  done_mask |= bit;
+  return true;
+}
+
 // Multiprocessor count of the current device (queried once per device).
 int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (cached[dev] == 0) {
@@ -166,7 +184,7 @@ int sm_count() {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
     cached[dev] = n;
   }
-  return cached[dev];
+  return cached[dev].load();
 }
 
 bool shape_ok(int B, int H, int N, int d) {
@@ -216,19 +234,13 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   cudaError_t e;
   if (o_hp == nullptr) {
     using L = fa::FwdLayout<D, false>;
-    static bool attr = false;
-    if (!attr) {
-      if (!set_smem(fa::fa_fwd_kernel<D, false>, L::SMEM_BYTES)) return FA_ERR_CUDA;
-      attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    if (!ensure_smem(fa::fa_fwd_kernel<D, false>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
     e = launch(fa::fa_fwd_kernel<D, false>, L::SMEM_BYTES, L::CTAS_PER_SM);
   } else {
     using L = fa::FwdLayout<D, true>;
-    static bool attr = false;
-    if (!attr) {
-      if (!set_smem(fa::fa_fwd_kernel<D, true>, L::SMEM_BYTES)) return FA_ERR_CUDA;
-      attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    if (!ensure_smem(fa::fa_fwd_kernel<D, true>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
     e = launch(fa::fa_fwd_kernel<D, true>, L::SMEM_BYTES, L::CTAS_PER_SM);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
@@ -248,14 +260,11 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      int causal, int mode, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
   using LP = fa::BwdPipeLayout;
-  static bool attr = false;
-  if (!attr) {
-    if (D == 64) {
-      if (!set_smem(fa::fa_bwd_main_pipe_kernel, LP::SMEM_BYTES)) return FA_ERR_CUDA;
-    } else {
-      if (!set_smem(fa::fa_bwd_main_kernel<D>, L::SMEM_BYTES)) return FA_ERR_CUDA;
-    }
-    attr = true;
+  static std::atomic<uint64_t> attr{0};
+  if (D == 64) {
+    if (!ensure_smem(fa::fa_bwd_main_pipe_kernel, LP::SMEM_BYTES, attr)) return FA_ERR_CUDA;
+  } else {
+    if (!ensure_smem(fa::fa_bwd_main_kernel<D>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
   }
   const long long rows = static_cast<long long>(BH) * N;
   float* delta = reinterpret_cast<float*>(ws);
@@ -477,6 +486,7 @@ fa_status fa_timing_enable(int enable) {
 
 fa_status fa_timing_read(int* launches, double* total_ms) {
   if (!launches || !total_ms) return FA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_timing_mutex);
   for (int i = 0; i < FA_NUM_KERNELS; ++i) {
     launches[i] = 0;
     total_ms[i] = 0.0;
