@@ -41,7 +41,7 @@ WORKLOAD = "g2s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ("bf16_numerics_b200/csrc/fa_ptx.cuh", "bf16_numerics_b200/csrc/fa_fwd.cuh",
                   "bf16_numerics_b200/csrc/fa_bwd.cuh", "bf16_numerics_b200/csrc/fa_bwd_pipe.cuh",
-                  "bf16_numerics_b200/csrc/fa_lib.cu")
+                  "bf16_numerics_b200/csrc/fa_bwd_pipe128.cuh", "bf16_numerics_b200/csrc/fa_lib.cu")
 
 
 def parse_args():

@@ -1,7 +1,7 @@
 // Persistent, pipelined backward main kernel for head dimension 64.
 //
-// Same mathematics as fa_bwd_main_kernel (see fa_bwd.cuh): the work is split
-// into items = (batch*head, 128-key block); an item loops over the query blocks
+// Mathematics and products as listed in fa_bwd.cuh: the work is split into
+// items = (batch*head, 128-key block); an item loops over the query blocks
 // that see its keys, in the transposed orientation (lane = key).  One CTA per
 // SM walks a list of items (snake order over the CTAs, items sorted by
 // decreasing work), so TMEM allocation and barrier set-up happen once per CTA

@@ -1,0 +1,527 @@
+// Persistent, pipelined backward main kernel for head dimension 128.
+//
+// Same mathematics and work items as the d = 64 kernel (fa_bwd_pipe.cuh): an
+// item is one 128-key block of one (batch, head), looping over the query
+// blocks that see its keys, in the transposed orientation (lane = key); one
+// CTA per SM walks its list of items (longest first, snake order over CTAs).
+//
+// At d = 128 the four 128-column TMEM regions S^T, dP^T, dV and dK fill all
+// 512 columns and shared memory holds one K/V pair, a two-deep Q/dO ring and
+// one dS tile, so the schedule differs from d = 64:
+//   * dQ_g = dS K (N = 128) goes into the dP^T columns, issued right after
+//     dK_g, which reads dS^T from those columns (products issued by one
+//     thread run in issue order).  dP^T of block g+1 waits until the drain
+//     warps have copied dQ_g out of TMEM.
+//   * S^T of block g+1 is issued right after dV_g (which reads P^T_g from
+//     the S^T columns), so the elementwise warps find it ready when they
+//     finish dS of block g, and dK_g, dQ_g, dP^T_g+1 run on the tensor cores
+//     while they compute P of block g+1.
+//   * Eight elementwise warps (two warpgroups) split the 128 query columns of
+//     a key row: warpgroup h takes columns [64h, 64h+64).  Both copy their S^T
+//     columns to registers and meet at a named barrier; then warpgroup h
+//     writes its bf16 P^T into S^T cols [32h, 32h+32).  dS^T goes into the
+//     first half of the dP^T columns each warpgroup has just read
+//     (64h + [0,32)), which needs no barrier, and as a 128B-swizzled tile into
+//     shared memory for dQ.
+//   * Each warpgroup publishes the per-query vectors (exponent offset, 1/l,
+//     delta) of its 64 query columns in shared memory at the top of a block,
+//     from values loaded one block ahead.
+//   * Four drain warps add the dQ partial (times the softmax scale) to the
+//     fp32 accumulator with red.global.add.v4, 64 columns at a time, and
+//     release the dP^T columns as soon as the last columns are in registers.
+//   * The elementwise warps also write dK and dV at the end of an item,
+//     straight from TMEM to global memory.
+//
+// Barrier phases count a global query-block index g that runs across the
+// CTA's items; every phase of every barrier is waited for in order and no
+// producer can get two phases ahead of a consumer's wait.
+//
+// TMEM columns: S^T [0,128)  dP^T / dQ [128,256)  dV [256,384)  dK [384,512)
+// Warps: 0-3 and 4-7 elementwise (key t = threadIdx % 128), 8-11 drain
+// (query t), 12 TMA producer, 13 MMA issuer / TMEM owner, 14-15 idle.  The
+// block is launched with 128 registers per thread; the warpgroups then
+// re-balance them: elementwise 168, drain 88, TMA/MMA 88
+// (2*168 + 88 + 88 = 512 = 4*128).
+#pragma once
+
+#include "fa_bwd_pipe.cuh"
+
+namespace fa {
+
+struct BwdPipe128Layout {
+  static constexpr int D = 128, B = 128, NST = 2;
+  static constexpr int HALF = 128 * 128;                 // one 64-column half of a tile (128 rows x 128 B)
+  static constexpr int TILE = 2 * HALF;                  // 128 rows x 128 bf16
+  static constexpr int K_OFF = 0, V_OFF = TILE, Q_OFF = 2 * TILE;
+  static constexpr int DO_OFF = Q_OFF + NST * TILE;
+  static constexpr int DS_OFF = DO_OFF + NST * TILE;     // dS^T [keys][queries], two 64-query halves
+  static constexpr int VEC_OFF = DS_OFF + TILE;          // [3][128] fp32: exponent offset, 1/l, delta
+  static constexpr int BAR_OFF = VEC_OFF + 3 * 128 * 4;
+  enum {
+    KV_FULL = 0,
+    KV_EMPTY,
+    Q_FULL,
+    Q_EMPTY = Q_FULL + NST,
+    S_FULL = Q_EMPTY + NST,
+    P_FULL,
+    DP_FULL,
+    DS_FULL,
+    DQ_FULL,
+    DQ_FREE,
+    ACC_DONE,
+    ACC_FREE,
+    TEARDOWN,
+    NBAR
+  };
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512, S_COL = 0, DP_COL = 128, DV_COL = 256, DK_COL = 384;
+  static constexpr int THREADS = 512;
+  static constexpr uint32_t REGS_ELEM = 168, REGS_DRAIN = 88, REGS_CTRL = 88;
+};
+static_assert(BwdPipe128Layout::SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+__global__ void __launch_bounds__(512, 1)
+fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                           const BwdParams p) {
+  using L = BwdPipe128Layout;
+  constexpr int TILE = L::TILE, HALF = L::HALF, NST = L::NST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+  auto bar = [&](int i) { return base + L::BAR_OFF + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  const BoundedWait wait{abort_flag, 4u};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::KV_FULL), 1);
+    mbar_init(bar(L::KV_EMPTY), 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar(L::Q_FULL + s), 1);
+      mbar_init(bar(L::Q_EMPTY + s), 1);
+    }
+    mbar_init(bar(L::S_FULL), 1);
+    mbar_init(bar(L::P_FULL), 256);
+    mbar_init(bar(L::DP_FULL), 1);
+    mbar_init(bar(L::DS_FULL), 256);
+    mbar_init(bar(L::DQ_FULL), 1);
+    mbar_init(bar(L::DQ_FREE), 128);
+    mbar_init(bar(L::ACC_DONE), 1);
+    mbar_init(bar(L::ACC_FREE), 256);
+    mbar_init(bar(L::TEARDOWN), 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 13) {
+    tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  grid_launch_dependents();
+  grid_dependency_wait();  // delta and the cleared dQ accumulator come from the previous grid
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // End of every role: all 16 warps meet on named barrier 15, then warp 13
+  // waits for its last MMAs and frees TMEM.
+  auto teardown = [&]() {
+    tc_fence_before();
+    named_barrier_sync(15, L::THREADS);
+    if (warp == 13) {
+      tc_fence_after();
+      volatile int never = 0;
+      const BoundedWait drain{&never, 4u};
+      drain(bar(L::TEARDOWN), 0, 30);
+      tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+  };
+
+  if (warp >= 12) {
+    warpgroup_reg_dealloc<L::REGS_CTRL>();
+    if (warp == 12 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      BwdCursor cur;
+      cur.start(p);
+      int g = 0, last_r = -1;
+      int issued[NST];
+      for (int s = 0; s < NST; ++s) issued[s] = -1;
+      auto load_q = [&](int i, int gq) {
+        const int s = gq % NST, use = gq / NST;
+        if (use > 0 && !wait(bar(L::Q_EMPTY + s), (use - 1) & 1, 1)) return false;
+        const int row0 = (cur.i0 + i) * L::B;
+        const uint32_t qd = base + L::Q_OFF + s * TILE, dod = base + L::DO_OFF + s * TILE;
+        mbar_expect_tx(bar(L::Q_FULL + s), 2 * TILE);
+        for (int h = 0; h < 2; ++h) {
+          tma_load_3d(qd + h * HALF, &tm_q, bar(L::Q_FULL + s), 64 * h, row0, cur.bh);
+          tma_load_3d(dod + h * HALF, &tm_do, bar(L::Q_FULL + s), 64 * h, row0, cur.bh);
+        }
+        issued[s] = gq;
+        return true;
+      };
+      bool ok = true;
+      for (; ok && cur.valid; cur.next_item()) {
+        // the item's first query block goes ahead of its K/V, which must wait
+        // for the previous item's products to release the K/V tiles; at the
+        // cold start the rest of the ring waits until the first products'
+        // operands (K, V, Q_0, dO_0) have arrived
+        ok = load_q(0, g);
+        if (!ok) break;
+        if (cur.r > 0 && !wait(bar(L::KV_EMPTY), (cur.r - 1) & 1, 1)) break;
+        mbar_expect_tx(bar(L::KV_FULL), 2 * TILE);
+        for (int h = 0; h < 2; ++h) {
+          tma_load_3d(base + L::K_OFF + h * HALF, &tm_k, bar(L::KV_FULL), 64 * h, cur.kblk * L::B, cur.bh);
+          tma_load_3d(base + L::V_OFF + h * HALF, &tm_v, bar(L::KV_FULL), 64 * h, cur.kblk * L::B, cur.bh);
+        }
+        last_r = cur.r;
+        if (cur.r == 0 && (!wait(bar(L::KV_FULL), 0, 23) || !wait(bar(L::Q_FULL), 0, 24))) break;
+        for (int i = 1; ok && i < cur.n; ++i) ok = load_q(i, g + i);
+        g += cur.n;
+      }
+      volatile int never = 0;
+      const BoundedWait drain{&never, 4u};
+      if (last_r >= 0) drain(bar(L::KV_FULL), last_r & 1, 20);
+      for (int s = 0; s < NST; ++s)
+        if (issued[s] >= 0) drain(bar(L::Q_FULL + s), (issued[s] / NST) & 1, 21);
+    } else if (warp == 13 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t IDESC_SQ = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
+      constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, false, true);   // dV, dK
+      constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, 128, true, true);    // dQ
+      auto q_tile = [&](int g) { return base + L::Q_OFF + (g % NST) * TILE; };
+      auto do_tile = [&](int g) { return base + L::DO_OFF + (g % NST) * TILE; };
+      // S^T = K Q_g^T and dP^T = V dO_g^T   (K-dim = d: two 64-column halves)
+      auto issue_s = [&](int g) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
+          mma_ss(tmem + L::S_COL, sdesc_sw128(base + L::K_OFF + koff, 16, 1024),
+                 sdesc_sw128(q_tile(g) + koff, 16, 1024), IDESC_SQ, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(L::S_FULL));
+      };
+      auto issue_dp = [&](int g) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
+          mma_ss(tmem + L::DP_COL, sdesc_sw128(base + L::V_OFF + koff, 16, 1024),
+                 sdesc_sw128(do_tile(g) + koff, 16, 1024), IDESC_SQ, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(L::DP_FULL));
+      };
+      BwdCursor cur;
+      cur.start(p);
+      int g = 0;
+      bool ok = true;
+      for (; ok && cur.valid; cur.next_item()) {
+        const int n = cur.n;
+        if (!wait(bar(L::KV_FULL), cur.r & 1, 2)) break;
+        // S^T and dP^T of the item's first block; dP^T waits for the drain
+        // of the previous block's dQ, which sits in the same columns
+        if (!wait(bar(L::Q_FULL + (g % NST)), (g / NST) & 1, 3)) break;
+        tc_fence_after();
+        issue_s(g);
+        if (g > 0 && !wait(bar(L::DQ_FREE), (g - 1) & 1, 6)) break;
+        tc_fence_after();
+        issue_dp(g);
+        for (int i = 0; i < n; ++i, ++g) {
+          if (!wait(bar(L::P_FULL), g & 1, 4)) { ok = false; break; }
+          // the first products of an item overwrite the accumulators: the
+          // previous item's epilogue must have copied them out
+          if (i == 0 && cur.r > 0 && !wait(bar(L::ACC_FREE), (cur.r - 1) & 1, 8)) { ok = false; break; }
+          tc_fence_after();
+          // dV += P^T dO_g   (K-dim = queries; P^T at S^T cols [0,64))
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ts(tmem + L::DV_COL, tmem + L::S_COL + 8u * ks, sdesc_sw128(do_tile(g) + ks * 2048, HALF, 1024),
+                   IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
+          // S^T of the next block overwrites P^T_g after dV_g has read it
+          if (i + 1 < n) {
+            if (!wait(bar(L::Q_FULL + ((g + 1) % NST)), ((g + 1) / NST) & 1, 3)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(g + 1);
+          }
+          if (!wait(bar(L::DS_FULL), g & 1, 5)) { ok = false; break; }
+          tc_fence_after();
+          // dK += dS^T Q_g   (dS^T at dP^T cols 64h + [0,32))
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t a = tmem + L::DP_COL + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4));
+            mma_ts(tmem + L::DK_COL, a, sdesc_sw128(q_tile(g) + ks * 2048, HALF, 1024), IDESC_KV,
+                   (i > 0 || ks > 0) ? 1u : 0u);
+          }
+          // dQ_g = dS K into the dP^T columns (after dK_g has read dS^T there)
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + L::DP_COL, sdesc_sw128(base + L::DS_OFF + ks * 2048, HALF, 1024),
+                   sdesc_sw128(base + L::K_OFF + ks * 2048, HALF, 1024), IDESC_DQ, ks > 0 ? 1u : 0u);
+          tc_commit(bar(L::DQ_FULL));
+          tc_commit(bar(L::Q_EMPTY + (g % NST)));
+          if (i + 1 == n) {
+            tc_commit(bar(L::ACC_DONE));  // dV, dK of this item complete
+            tc_commit(bar(L::KV_EMPTY));  // K, V of this item no longer read
+          } else {
+            if (!wait(bar(L::DQ_FREE), g & 1, 6)) { ok = false; break; }
+            tc_fence_after();
+            issue_dp(g + 1);
+          }
+        }
+      }
+      tc_commit(bar(L::TEARDOWN));
+    }
+    __syncwarp();
+    teardown();
+    return;
+  }
+
+  if (warp >= 8) {
+    warpgroup_reg_dealloc<L::REGS_DRAIN>();
+    // ----------------------------------------------------------- drain warps
+    const int t = threadIdx.x - 256;  // query within the block == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float scale = p.scale;
+    BwdCursor cur;
+    cur.start(p);
+    for (int g = 0; cur.valid; ++g, cur.next_block()) {
+      // a wait that gives up ends the loop (the reads below would be stale)
+      if (!wait.warp(bar(L::DQ_FULL), g & 1, 13)) break;
+      tc_fence_after();
+      const int q_row = cur.qblk() * L::B + t;
+      const bool row_ok = q_row < p.N;
+      float* dst = p.dq_acc + (static_cast<size_t>(cur.bh) * p.N + (row_ok ? q_row : 0)) * L::D;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32x2(tmem + lane_base + L::DP_COL + 64u * half, tmem + lane_base + L::DP_COL + 64u * half + 32u, r0,
+                    r1);
+        if (half == 1) {
+          tc_fence_before();
+          mbar_arrive(bar(L::DQ_FREE));  // dP^T of the next block may overwrite the columns
+        }
+        if (row_ok) {
+          float* d = dst + 64 * half;
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            red_add_v4(d + c, __uint_as_float(r0[c]) * scale, __uint_as_float(r0[c + 1]) * scale,
+                       __uint_as_float(r0[c + 2]) * scale, __uint_as_float(r0[c + 3]) * scale);
+            red_add_v4(d + 32 + c, __uint_as_float(r1[c]) * scale, __uint_as_float(r1[c + 1]) * scale,
+                       __uint_as_float(r1[c + 2]) * scale, __uint_as_float(r1[c + 3]) * scale);
+          }
+        }
+      }
+    }
+    teardown();
+    return;
+  }
+
+  {
+    warpgroup_reg_alloc<L::REGS_ELEM>();
+    // ------------------------------------------------- elementwise warps 0..7
+    const int h = warp >> 2;          // query half
+    const int t = threadIdx.x & 127;  // key within the block == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float scale = p.scale;
+    const float c_log2 = scale * kLog2e;
+    const uint64_t C2 = f2_pack(c_log2, c_log2);
+    const bool mode1 = p.mode == 1;
+    const int qoff = 64 * h;
+    const uint32_t ds_row = base + L::DS_OFF + h * HALF + t * 128;
+    const uint32_t va = base + L::VEC_OFF + (0 * 128 + qoff) * 4;
+    const uint32_t vb = base + L::VEC_OFF + (1 * 128 + qoff) * 4;
+    const uint32_t vd = base + L::VEC_OFF + (2 * 128 + qoff) * 4;
+    // Per-query vectors: thread t publishes query 64h + (t & 63) of the block,
+    // threads t < 64 the exponent offset and 1/l, threads t >= 64 delta.  The
+    // raw values are loaded one block ahead (cursor pf).
+    const int vq = t & 63, vrole = t >> 6;
+    BwdCursor pf;
+    pf.start(p);
+    auto fetch = [&](float& x, float& y) {
+      x = 0.f;
+      y = 0.f;
+      if (pf.valid) {
+        const int q = pf.qblk() * L::B + qoff + vq;
+        if (q < p.N) {
+          const size_t vi = static_cast<size_t>(pf.bh) * p.N + q;
+          if (vrole == 0) {
+            x = __ldg(p.lse + vi);
+            y = mode1 ? __ldg(p.row_m + vi) : 0.f;
+          } else {
+            x = __ldg(p.delta + vi);
+          }
+        } else {
+          x = INFINITY;  // padded query: P = 0
+        }
+      }
+      pf.next_block();
+    };
+    float nx, ny;
+    fetch(nx, ny);
+    BwdCursor cur;
+    cur.start(p);
+    int g = 0;
+    // Error discipline as in the d = 64 kernel: the two warpgroups meet on
+    // named barrier 1 once per block (an AND vote); a bounded wait that gives
+    // up only clears `ok`, and the next vote takes both warpgroups out.
+    bool ok = true;
+    for (; cur.valid; cur.next_item()) {
+      bool leave = false;
+      for (int i = 0; i < cur.n; ++i, ++g) {
+        // this warpgroup has finished with the previous block's vectors
+        named_barrier_sync(3 + h, 128);
+        if (vrole == 0) {
+          float na, bb;
+          if (nx == INFINITY) {
+            na = -INFINITY;
+            bb = 0.f;
+          } else if (mode1) {
+            na = -ny * kLog2e;
+            bb = 1.f / ex2_approx((nx - ny) * kLog2e);
+          } else {
+            na = -nx * kLog2e;
+            bb = 1.f;
+          }
+          sts32(va + vq * 4, na);
+          sts32(vb + vq * 4, bb);
+        } else {
+          sts32(vd + vq * 4, nx == INFINITY ? 0.f : nx);
+        }
+        fetch(nx, ny);
+        ok = ok && wait.warp(bar(L::S_FULL), g & 1, 9);
+        tc_fence_after();
+        const bool diag = p.causal && (cur.i0 + i == cur.kblk);
+        uint64_t p2[32];  // this row's 64 P values (fp32 pairs)
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32x2(tmem + lane_base + L::S_COL + 64u * h, tmem + lane_base + L::S_COL + 64u * h + 32u, r0, r1);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            p2[e] = f2_pack(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
+            p2[16 + e] = f2_pack(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+          }
+        }
+        // both warpgroups hold their S^T columns (P^T may now overwrite
+        // [0,64)) and have published their vectors
+        if (!named_barrier_and(1, 256, ok)) { leave = true; break; }
+        uint32_t pk[32];
+#pragma unroll
+        for (int pi = 0; pi < 32; pi += 2) {
+          const int ql = 2 * pi;
+          const float4 na = lds128(va + ql * 4);
+          const uint64_t y0 = f2_fma(p2[pi], C2, f2_pack(na.x, na.y));
+          const uint64_t y1 = f2_fma(p2[pi + 1], C2, f2_pack(na.z, na.w));
+          float a0, a1, a2, a3;
+          f2_unpack(y0, a0, a1);
+          f2_unpack(y1, a2, a3);
+          float p0 = ex2_approx(a0), p1 = ex2_approx(a1), p2v = ex2_approx(a2), p3 = ex2_approx(a3);
+          if (mode1) {
+            const float4 bb = lds128(vb + ql * 4);
+            p0 *= bb.x;
+            p1 *= bb.y;
+            p2v *= bb.z;
+            p3 *= bb.w;
+          }
+          if (diag) {
+            const int qg = qoff + ql;
+            if (t > qg) p0 = 0.f;
+            if (t > qg + 1) p1 = 0.f;
+            if (t > qg + 2) p2v = 0.f;
+            if (t > qg + 3) p3 = 0.f;
+          }
+          p2[pi] = f2_pack(p0, p1);
+          p2[pi + 1] = f2_pack(p2v, p3);
+          pk[pi] = pack_bf16x2(p0, p1);
+          pk[pi + 1] = pack_bf16x2(p2v, p3);
+        }
+        tmem_st32(tmem + lane_base + L::S_COL + 32u * h, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::P_FULL));
+        // dP^T of this block; it is issued after the previous block's dQ
+        // product has completed, so the dS tile in shared memory is free too
+        ok = wait.warp(bar(L::DP_FULL), g & 1, 10);
+        if (!ok) continue;  // the next meeting takes everyone out
+        tc_fence_after();
+        uint32_t dpr[64];
+        {
+          uint32_t(&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]);
+          uint32_t(&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]);
+          tmem_ld32x2(tmem + lane_base + L::DP_COL + 64u * h, tmem + lane_base + L::DP_COL + 64u * h + 32u, d0, d1);
+        }
+        uint32_t dk_[32];
+#pragma unroll
+        for (int pi = 0; pi < 32; pi += 2) {
+          const int ql = 2 * pi;
+          const float4 dl = lds128(vd + ql * 4);
+          const uint64_t ds0 = f2_mul(
+              p2[pi], f2_sub(f2_pack(__uint_as_float(dpr[2 * pi]), __uint_as_float(dpr[2 * pi + 1])), f2_pack(dl.x, dl.y)));
+          const uint64_t ds1 =
+              f2_mul(p2[pi + 1], f2_sub(f2_pack(__uint_as_float(dpr[2 * pi + 2]), __uint_as_float(dpr[2 * pi + 3])),
+                                        f2_pack(dl.z, dl.w)));
+          float d0, d1, d2, d3;
+          f2_unpack(ds0, d0, d1);
+          f2_unpack(ds1, d2, d3);
+          dk_[pi] = pack_bf16x2(d0, d1);
+          dk_[pi + 1] = pack_bf16x2(d2, d3);
+        }
+        // dS^T into the dP^T columns this warpgroup has read: 64h + [0,32)
+        tmem_st32(tmem + lane_base + L::DP_COL + 64u * h, dk_);
+        // dS^T row t, queries 64h + [0,64) = the eight 16-byte chunks of the half tile's row
+#pragma unroll
+        for (int chunk = 0; chunk < 8; ++chunk)
+          sts128(ds_row + ((chunk ^ (t & 7)) << 4), dk_[4 * chunk], dk_[4 * chunk + 1], dk_[4 * chunk + 2],
+                 dk_[4 * chunk + 3]);
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::DS_FULL));
+      }
+      if (leave) break;
+      // ----------------------------------------------------- item epilogue
+      // warpgroup 0 writes dV, warpgroup 1 writes dK * scale: TMEM -> bf16
+      // -> global memory, one 256-byte row per thread (rows past N skipped)
+      ok = ok && wait.warp(bar(L::ACC_DONE), cur.r & 1, 12);
+      tc_fence_after();
+      const float f = (h == 0) ? 1.f : scale;
+      const uint32_t col = (h == 0) ? L::DV_COL : L::DK_COL;
+      const int key = cur.kblk * L::B + t;
+      const bool row_ok = ok && key < p.N;
+      __nv_bfloat16* dst = (h == 0 ? p.dv : p.dk) + (static_cast<size_t>(cur.bh) * p.N + (row_ok ? key : 0)) * L::D;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32x2(tmem + lane_base + col + 64u * half, tmem + lane_base + col + 64u * half + 32u, r0, r1);
+        if (half == 1) {
+          tc_fence_before();
+          mbar_arrive(bar(L::ACC_FREE));  // the next item may overwrite the accumulators
+        }
+        if (row_ok) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            uint4 w0, w1;
+            w0.x = pack_bf16x2(__uint_as_float(r0[c + 0]) * f, __uint_as_float(r0[c + 1]) * f);
+            w0.y = pack_bf16x2(__uint_as_float(r0[c + 2]) * f, __uint_as_float(r0[c + 3]) * f);
+            w0.z = pack_bf16x2(__uint_as_float(r0[c + 4]) * f, __uint_as_float(r0[c + 5]) * f);
+            w0.w = pack_bf16x2(__uint_as_float(r0[c + 6]) * f, __uint_as_float(r0[c + 7]) * f);
+            w1.x = pack_bf16x2(__uint_as_float(r1[c + 0]) * f, __uint_as_float(r1[c + 1]) * f);
+            w1.y = pack_bf16x2(__uint_as_float(r1[c + 2]) * f, __uint_as_float(r1[c + 3]) * f);
+            w1.z = pack_bf16x2(__uint_as_float(r1[c + 4]) * f, __uint_as_float(r1[c + 5]) * f);
+            w1.w = pack_bf16x2(__uint_as_float(r1[c + 6]) * f, __uint_as_float(r1[c + 7]) * f);
+            *reinterpret_cast<uint4*>(dst + 64 * half + c) = w0;
+            *reinterpret_cast<uint4*>(dst + 64 * half + 32 + c) = w1;
+          }
+        }
+      }
+    }
+    teardown();
+  }
+}
+
+}  // namespace fa

@@ -15,6 +15,7 @@
 
 #include "fa_b200.h"
 #include "fa_bwd_pipe.cuh"
+#include "fa_bwd_pipe128.cuh"
 
 namespace {
 
@@ -258,13 +259,13 @@ template <int D>
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, bool o_is_hp, const void* dO,
                      const float* lse, const float* row_m, void* dq, void* dk, void* dv, uint8_t* ws, int BH, int N,
                      int causal, int mode, cudaStream_t stream) {
-  using L = fa::BwdLayout<D>;
   using LP = fa::BwdPipeLayout;
+  using LP128 = fa::BwdPipe128Layout;
   static std::atomic<uint64_t> attr{0};
   if (D == 64) {
     if (!ensure_smem(fa::fa_bwd_main_pipe_kernel, LP::SMEM_BYTES, attr)) return FA_ERR_CUDA;
   } else {
-    if (!ensure_smem(fa::fa_bwd_main_kernel<D>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
+    if (!ensure_smem(fa::fa_bwd_main_pipe128_kernel, LP128::SMEM_BYTES, attr)) return FA_ERR_CUDA;
   }
   const long long rows = static_cast<long long>(BH) * N;
   float* delta = reinterpret_cast<float*>(ws);
@@ -301,12 +302,12 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.causal = causal;
     p.mode = mode;
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    // persistent: one CTA per SM (at most one per work item)
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_blk) * BH);
+    const int n_sm = sm_count();
+    if (n_sm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)");
+    const unsigned pgrid = grid < static_cast<unsigned>(n_sm) ? grid : static_cast<unsigned>(n_sm);
     if (D == 64) {
-      // persistent: one CTA per SM (at most one per work item)
-      const int n_sm = sm_count();
-      if (n_sm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)");
-      const unsigned pgrid = grid < static_cast<unsigned>(n_sm) ? grid : static_cast<unsigned>(n_sm);
       CUtensorMap mdq, mdk, mdv;
       if (!make_map_dq(&mdq, dq_acc, BH, N)) return cuda_fail("cuTensorMapEncodeTiled (dQ accumulator)");
       if (!make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
@@ -319,8 +320,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
     } else {
       LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
-      cudaError_t e = launch_pdl(fa::fa_bwd_main_kernel<D>, dim3(grid), dim3(320), L::SMEM_BYTES, stream, mq, mk, mv,
-                                 mdo, p);
+      cudaError_t e = launch_pdl(fa::fa_bwd_main_pipe128_kernel, dim3(pgrid), dim3(LP128::THREADS),
+                                 LP128::SMEM_BYTES, stream, mq, mk, mv, mdo, p);
       tm.done();
       if (e == cudaSuccess) e = cudaGetLastError();
       if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
