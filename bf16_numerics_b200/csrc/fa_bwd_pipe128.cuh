@@ -27,8 +27,12 @@
 //     delta) of its 64 query columns in shared memory at the top of a block,
 //     from values loaded one block ahead.
 //   * Four drain warps add the dQ partial (times the softmax scale) to the
-//     fp32 accumulator with red.global.add.v4, 64 columns at a time, and
-//     release the dP^T columns as soon as the last columns are in registers.
+//     fp32 accumulator with TMA tensor reduce-adds, 64 columns at a time,
+//     staged as two 128B-swizzled [128 rows][32 fp32] boxes in the dS tile
+//     (free from the end of dQ_g until the elementwise warps write dS of the
+//     next block, which they do only after the drain has released it).  The
+//     dP^T columns are released as soon as the last dQ columns are in
+//     registers.
 //   * The elementwise warps also write dK and dV at the end of an item,
 //     straight from TMEM to global memory.
 //
@@ -70,6 +74,7 @@ struct BwdPipe128Layout {
     DQ_FREE,
     ACC_DONE,
     ACC_FREE,
+    DSTILE_FREE,  // the drain's reduce-adds have read the dS tile
     TEARDOWN,
     NBAR
   };
@@ -84,7 +89,7 @@ static_assert(BwdPipe128Layout::SMEM_BYTES <= 227 * 1024, "shared memory budget"
 __global__ void __launch_bounds__(512, 1)
 fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                           const BwdParams p) {
+                           const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using L = BwdPipe128Layout;
   constexpr int TILE = L::TILE, HALF = L::HALF, NST = L::NST;
   extern __shared__ uint8_t smem_raw[];
@@ -112,6 +117,7 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
     mbar_init(bar(L::DQ_FREE), 128);
     mbar_init(bar(L::ACC_DONE), 1);
     mbar_init(bar(L::ACC_FREE), 256);
+    mbar_init(bar(L::DSTILE_FREE), 1);
     mbar_init(bar(L::TEARDOWN), 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -288,36 +294,62 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
     const int t = threadIdx.x - 256;  // query within the block == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float scale = p.scale;
+    if (t == 0) tma_prefetch_desc(&tm_dq);
     BwdCursor cur;
     cur.start(p);
+    // A bounded wait that gives up only clears `ok`; the warpgroup leaves the
+    // loop together at the AND vote on named barrier 2.
+    bool ok = true;
+    // row t of a [128][32 fp32] box, 16-byte chunk c stored at chunk c ^ (t & 7)
+    auto stage = [&](uint32_t box, const uint32_t (&r)[32]) {
+      const uint32_t row = box + t * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        sts128(row + ((c ^ (t & 7)) << 4), __float_as_uint(__uint_as_float(r[4 * c]) * scale),
+               __float_as_uint(__uint_as_float(r[4 * c + 1]) * scale),
+               __float_as_uint(__uint_as_float(r[4 * c + 2]) * scale),
+               __float_as_uint(__uint_as_float(r[4 * c + 3]) * scale));
+    };
+    const uint32_t box0 = base + L::DS_OFF, box1 = base + L::DS_OFF + HALF;
     for (int g = 0; cur.valid; ++g, cur.next_block()) {
-      // a wait that gives up ends the loop (the reads below would be stale)
-      if (!wait.warp(bar(L::DQ_FULL), g & 1, 13)) break;
+      {
+        // every lane calls the warp-uniform wait (ok may differ per lane here)
+        const bool got = wait.warp(bar(L::DQ_FULL), g & 1, 13);
+        ok = ok && got;
+      }
       tc_fence_after();
-      const int q_row = cur.qblk() * L::B + t;
-      const bool row_ok = q_row < p.N;
-      float* dst = p.dq_acc + (static_cast<size_t>(cur.bh) * p.N + (row_ok ? q_row : 0)) * L::D;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t r0[32], r1[32];
-        tmem_ld32x2(tmem + lane_base + L::DP_COL + 64u * half, tmem + lane_base + L::DP_COL + 64u * half + 32u, r0,
-                    r1);
-        if (half == 1) {
-          tc_fence_before();
-          mbar_arrive(bar(L::DQ_FREE));  // dP^T of the next block may overwrite the columns
-        }
-        if (row_ok) {
-          float* d = dst + 64 * half;
-#pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            red_add_v4(d + c, __uint_as_float(r0[c]) * scale, __uint_as_float(r0[c + 1]) * scale,
-                       __uint_as_float(r0[c + 2]) * scale, __uint_as_float(r0[c + 3]) * scale);
-            red_add_v4(d + 32 + c, __uint_as_float(r1[c]) * scale, __uint_as_float(r1[c + 1]) * scale,
-                       __uint_as_float(r1[c + 2]) * scale, __uint_as_float(r1[c + 3]) * scale);
-          }
-        }
+      const int q0 = cur.qblk() * L::B;
+      uint32_t r0[32], r1[32];
+      // columns [0,64): the dS tile is free (dQ_g, its last reader, has completed)
+      tmem_ld32x2(tmem + lane_base + L::DP_COL, tmem + lane_base + L::DP_COL + 32u, r0, r1);
+      stage(box0, r0);
+      stage(box1, r1);
+      fence_proxy_async_smem();
+      if (!named_barrier_and(2, 128, ok)) break;
+      if (t == 0) {
+        tma_reduce_add_3d(&tm_dq, box0, 0, q0, cur.bh);
+        tma_reduce_add_3d(&tm_dq, box1, 32, q0, cur.bh);
+        bulk_commit();
+      }
+      // columns [64,128); then dP^T of the next block may overwrite them
+      tmem_ld32x2(tmem + lane_base + L::DP_COL + 64u, tmem + lane_base + L::DP_COL + 96u, r0, r1);
+      tc_fence_before();
+      mbar_arrive(bar(L::DQ_FREE));
+      if (t == 0) bulk_wait_read_all();  // the first two boxes have been read
+      named_barrier_sync(2, 128);
+      stage(box0, r0);
+      stage(box1, r1);
+      fence_proxy_async_smem();
+      named_barrier_sync(2, 128);
+      if (t == 0) {
+        tma_reduce_add_3d(&tm_dq, box0, 64, q0, cur.bh);
+        tma_reduce_add_3d(&tm_dq, box1, 96, q0, cur.bh);
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(bar(L::DSTILE_FREE));  // the elementwise warps may write dS again
       }
     }
+    if (t == 0) bulk_wait_all();
     teardown();
     return;
   }
@@ -444,8 +476,6 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(L::P_FULL));
-        // dP^T of this block; it is issued after the previous block's dQ
-        // product has completed, so the dS tile in shared memory is free too
         ok = wait.warp(bar(L::DP_FULL), g & 1, 10);
         if (!ok) continue;  // the next meeting takes everyone out
         tc_fence_after();
@@ -473,11 +503,18 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
         }
         // dS^T into the dP^T columns this warpgroup has read: 64h + [0,32)
         tmem_st32(tmem + lane_base + L::DP_COL + 64u * h, dk_);
+        // the dS tile also stages the previous block's dQ for the drain's
+        // reduce-adds: wait until they have read it (after a wait that gave
+        // up, skip the write; the next vote takes everyone out)
+        const bool tile_free = g == 0 || wait.warp(bar(L::DSTILE_FREE), (g - 1) & 1, 14);
+        ok = ok && tile_free;
         // dS^T row t, queries 64h + [0,64) = the eight 16-byte chunks of the half tile's row
+        if (tile_free) {
 #pragma unroll
-        for (int chunk = 0; chunk < 8; ++chunk)
-          sts128(ds_row + ((chunk ^ (t & 7)) << 4), dk_[4 * chunk], dk_[4 * chunk + 1], dk_[4 * chunk + 2],
-                 dk_[4 * chunk + 3]);
+          for (int chunk = 0; chunk < 8; ++chunk)
+            sts128(ds_row + ((chunk ^ (t & 7)) << 4), dk_[4 * chunk], dk_[4 * chunk + 1], dk_[4 * chunk + 2],
+                   dk_[4 * chunk + 3]);
+        }
         fence_proxy_async_smem();
         tmem_st_wait();
         tc_fence_before();

@@ -53,13 +53,13 @@ bool make_map(CUtensorMap* map, const void* ptr, long long BH, long long N, int 
   return r == CUDA_SUCCESS;
 }
 
-// fp32 dQ accumulator [BH, N, 64] -> 3-D tensor map, box 32 (d) x 128 (rows) x 1,
+// fp32 dQ accumulator [BH, N, D] -> 3-D tensor map, box 32 (d) x 128 (rows) x 1,
 // 128B swizzle: the target of the pipelined backward's TMA reduce-add.
-bool make_map_dq(CUtensorMap* map, const void* ptr, long long BH, long long N) {
+bool make_map_dq(CUtensorMap* map, const void* ptr, long long BH, long long N, int D) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {64 * 4, static_cast<cuuint64_t>(N) * 64 * 4};
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(N) * D * 4};
   cuuint32_t box[3] = {32, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -302,14 +302,15 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.causal = causal;
     p.mode = mode;
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    CUtensorMap mdq;
+    if (!make_map_dq(&mdq, dq_acc, BH, N, D)) return cuda_fail("cuTensorMapEncodeTiled (dQ accumulator)");
     // persistent: one CTA per SM (at most one per work item)
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(p.n_blk) * BH);
     const int n_sm = sm_count();
     if (n_sm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)");
     const unsigned pgrid = grid < static_cast<unsigned>(n_sm) ? grid : static_cast<unsigned>(n_sm);
     if (D == 64) {
-      CUtensorMap mdq, mdk, mdv;
-      if (!make_map_dq(&mdq, dq_acc, BH, N)) return cuda_fail("cuTensorMapEncodeTiled (dQ accumulator)");
+      CUtensorMap mdk, mdv;
       if (!make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
         return cuda_fail("cuTensorMapEncodeTiled (dk/dv)");
       LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
@@ -321,7 +322,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     } else {
       LaunchTimer tm(FA_KERNEL_BWD_MAIN, stream);
       cudaError_t e = launch_pdl(fa::fa_bwd_main_pipe128_kernel, dim3(pgrid), dim3(LP128::THREADS),
-                                 LP128::SMEM_BYTES, stream, mq, mk, mv, mdo, p);
+                                 LP128::SMEM_BYTES, stream, mq, mk, mv, mdo, mdq, p);
       tm.done();
       if (e == cudaSuccess) e = cudaGetLastError();
       if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
