@@ -163,9 +163,10 @@ def test_margin_mode_small_ties(cuda_device, causal):
             assert np.all(gpu["m"][small] == gpu["rm"][small] + np.float32(2.0 ** -8))
 
 
-def test_empty_problem_is_noop(cuda_device):
+@pytest.mark.parametrize("d", [64, 128])
+def test_empty_problem_is_noop(cuda_device, d):
     import bf16_numerics_b200 as fa
-    q = torch.empty(1, 2, 0, 64, device=cuda_device, dtype=torch.bfloat16)
+    q = torch.empty(1, 2, 0, d, device=cuda_device, dtype=torch.bfloat16)
     o, lse, st = fa.attention_forward(q, q, q, True, 1, 2.0)
     assert o.numel() == 0
     dq, dk, dv, ws = fa.attention_backward(q, q, q, o, q, lse, st.m, True, 1, 2.0,
@@ -173,14 +174,36 @@ def test_empty_problem_is_noop(cuda_device):
     assert dq.numel() == 0
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("N", [1, 7, 129])
-def test_tiny_lengths(cuda_device, N):
+def test_tiny_lengths(cuda_device, N, d):
     """Lengths below and just above one tile."""
-    w = workloads.make("g2s", B=1, H=1, N=N, seed=N)
+    if d == 64:
+        w = workloads.make("g2s", B=1, H=1, N=N, seed=N)
+    else:
+        rng = np.random.default_rng(1000 + N)
+        mk = lambda: workloads.to_bf16_values(rng.standard_normal((1, 1, N, 128)).astype(np.float32))
+        w = workloads.Workload("d128", 1, 1, N, 128, True, 0, mk(), mk(), mk(), mk(), np.zeros((1, 1, N), bool))
     for mode in (0, 1):
         gpu = P.run_gpu(w, mode)
         ref = P.oracle(w, mode, o_gpu=gpu["o"])
         P.compare(gpu, ref, exact_stats=False)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_d128_several_items_per_cta(cuda_device, causal):
+    """More work items (key blocks x heads) than SMs at d = 128, compared on
+    every head: each persistent CTA of the backward walks several items, so
+    the K/V reloads, the accumulator hand-over between items and the dQ
+    reduce-adds from different CTAs into the same query block are exercised."""
+    rng = np.random.default_rng(4242)
+    B, H, N = 2, 48, 256 + 40
+    mk = lambda: workloads.to_bf16_values(rng.standard_normal((B, H, N, 128)).astype(np.float32))
+    w = workloads.Workload("d128", B, H, N, 128, causal, 0, mk(), mk(), mk(), mk(), np.zeros((B, H, N), bool))
+    assert B * H * ((N + 127) // 128) > 148
+    gpu = P.run_gpu(w, 1)
+    ref = P.oracle(w, 1, o_gpu=gpu["o"])
+    P.compare(gpu, ref, exact_stats=False)
 
 
 # ------------------------------------------------- full-size workloads (sampled)
