@@ -77,9 +77,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources (matching source hash); else None."""
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from a committed ncu
+    summary, if it was taken on the current kernel sources (matching source
+    hash); else None.  Line format: kernel workload source_hash bytes N."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
@@ -87,8 +88,9 @@ def recorded_traffic(kernel: str):
     with open(path) as f:
         for line in f:
             parts = line.split()
-            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == src:
-                return float(parts[3])
+            if (len(parts) >= 5 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload
+                    and parts[2] == src):
+                return float(parts[4])
     return None
 
 
@@ -439,7 +441,7 @@ def run_ours(args, rank, world, local_rank):
         kern[name]["launches"] = n_l
     dominant = max(per_kernel, key=lambda nm: per_kernel[nm][1])
     dk_ = kern[dominant]
-    traffic = recorded_traffic(dominant)
+    traffic = recorded_traffic(dominant, args.workload)
     roofline = {"kernel": dominant, "bound": dk_["bound"], "achieved": dk_["achieved"],
                 "peak": peak_tf if dk_["bound"] == "tensor" else hbm, "unit": dk_["unit"], "frac": dk_["frac"],
                 "traffic": traffic, "peak_source": f"{peak_src} ({'bf16_tflops burst' if dk_['bound'] == 'tensor' else 'hbm_gbs'})"}
