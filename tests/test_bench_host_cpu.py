@@ -1,0 +1,81 @@
+"""Host-side logic of bench.py on the CPU: the per-workload DRAM traffic
+record, the clock/throttle-reason parsing and the peaks fallback."""
+
+import os
+
+import bench
+
+
+def test_traffic_record_is_keyed_by_kernel_workload_and_sources(tmp_path, monkeypatch):
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.txt").write_text(
+        "# kernel workload source_hash unit bytes\n"
+        "fa_bwd_main_kernel g2s abc123 bytes 1000\n"
+        "fa_bwd_main_kernel long abc123 bytes 5000\n"
+        "fa_fwd_kernel g2s oldhash bytes 7\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc123")
+    assert bench.recorded_traffic("fa_bwd_main_kernel", "g2s") == 1000.0
+    assert bench.recorded_traffic("fa_bwd_main_kernel", "long") == 5000.0
+    assert bench.recorded_traffic("fa_bwd_main_kernel", "tiestress") is None  # no capture for it
+    assert bench.recorded_traffic("fa_fwd_kernel", "g2s") is None  # taken on other sources
+
+
+def test_traffic_record_missing_file(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("fa_bwd_main_kernel", "g2s") is None
+
+
+def test_committed_traffic_lines_parse():
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles", "traffic.txt")
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        kernel, workload, src, unit, value = line.split()
+        assert unit == "bytes" and float(value) > 0 and len(src) == 16
+        assert workload in ("g2s", "g2m", "tiestress", "long", "tiny")
+
+
+class _FakeProc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+
+def _sampler(lines):
+    s = bench.ClockSampler(0)
+    s.proc = _FakeProc()
+    s.lines = lines
+    return s
+
+
+def test_clock_sampler_reports_median_and_active_reasons():
+    lines = [
+        "1965, 1965, 450.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "1950, 1965, 610.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "1965, 1965, 500.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ]
+    r = _sampler(lines).stop()
+    assert r["sm_mhz"] == 1965.0 and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["sw_power_cap"]
+    assert r["samples"] == 3 and r["power_w_max"] == 610.0
+
+
+def test_clock_sampler_flags_slowdowns():
+    lines = ["1200, 1965, 300.0, 0x8, Active, Not Active, Active, Not Active"]
+    r = _sampler(lines).stop()
+    assert r["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+
+
+def test_clock_sampler_without_samples():
+    assert _sampler([]).stop()["reasons"] == ["no samples"]
+
+
+def test_peaks_fall_back_when_the_file_is_missing(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, src = bench.load_peaks()
+    assert src == "fallback"
+    assert peaks == bench.FALLBACK_PEAKS
