@@ -273,8 +273,6 @@ def test_o_for_delta_changes_only_delta_path():
     assert not np.array_equal(b_bf["delta"], b_ref["delta"])
 
 
-# ------------------------------------------------------- planted mistakes
-
 # ------------------------------------------------ margin variant (mode 2)
 
 def _small_tie_rows():
@@ -329,6 +327,10 @@ def test_margin_sweep_over_tied_maxima():
         ok = np.isfinite(pmax) & (pmax > 0)
         assert np.all(bf16.round_bf16(pmax[ok]) < 1.0)
 
+
+# ------------------------------------------------------- planted mistakes
+# Each test plants one plausible slip in the oracle (on the CPU) and checks
+# that a pin above would catch it.
 
 def test_planted_mistake_dropped_scale_is_caught(monkeypatch):
     monkeypatch.setattr(A, "scale_f64", lambda d: 1.0)
@@ -390,3 +392,35 @@ def test_planted_mistake_dropped_delta_is_caught():
     lm = float((A.attention_fwd(x, k, v, True, 1)["o"] * do).sum())
     fd = (lp - lm) / (2 * h)
     assert abs(b_wrong["dq"][0, 0, 3, 1] - fd) > 1e-4
+
+
+def test_planted_mistake_flipped_causal_mask_is_caught(monkeypatch):
+    """Keys after the query visible instead of keys before it: the brute-force
+    softmax (key j <= query i) disagrees."""
+    monkeypatch.setattr(A, "_mask", lambda n, causal: np.triu(np.ones((n, n), bool)) if causal
+                        else np.ones((n, n), bool))
+    rng = np.random.default_rng(21)
+    q, k, v = (_rand_bf16(rng, (1, 1, 8, 16)) for _ in range(3))
+    out = A.attention_fwd(q, k, v, True, 1)
+    o_ref, _ = _brute_fwd(q[0, 0], k[0, 0], v[0, 0], True)
+    assert not np.allclose(out["o"][0, 0], o_ref, rtol=1e-6)
+
+
+def test_planted_mistake_tie_count_of_one_is_caught(monkeypatch):
+    """A tie count that never exceeds 1 (the equality test dropped) leaves the
+    shift on the row maximum: the exact ones the fix must remove come back on
+    the tied rows of the tiny workload."""
+    real = A.row_stats
+
+    def no_ties(s32, mode, beta):
+        rm, rs, _ = real(s32, mode, beta)
+        rs = np.minimum(rs, 1).astype(np.int32)
+        return rm, rs, A.select_shift(rm, rs, beta, mode)
+
+    w = workloads.make("tiny")
+    tied = A.attention_fwd(w.q, w.k, w.v, True, 1)["rs"] > 1
+    monkeypatch.setattr(A, "row_stats", no_ties)
+    f = A.attention_fwd(w.q, w.k, w.v, True, 1, return_pbar=True)
+    assert tied.any()
+    assert np.all(f["pbar"].max(axis=-1)[tied] == 1.0)  # the fix's pin (max P_bar < 1) fails
+
