@@ -28,7 +28,8 @@ STABILIZED_MARGIN = _abi.FA_SOFTMAX_STABILIZED_MARGIN
 
 __all__ = ["FaError", "STANDARD", "STABILIZED", "STABILIZED_MARGIN", "RowStats", "fa_fwd", "fa_bwd", "fa_fwd_o_hp", "fa_bwd_o_hp", "fa_bwd_workspace_bytes",
            "fa_bwd_workspace_offsets", "fa_status_string", "fa_device_error", "fa_timing_enable",
-           "fa_timing_read", "attention_forward", "attention_backward", "library_path"]
+           "fa_timing_read", "fa_debug_set_wait_limit_ns", "fa_debug_inject_stall", "attention_forward",
+           "attention_backward", "library_path"]
 
 
 class FaError(RuntimeError):
@@ -188,6 +189,20 @@ def fa_device_error() -> tuple[int, int]:
     word = ctypes.c_uint(0)
     code = _abi.load().fa_device_error(ctypes.byref(word))
     return int(code), int(word.value)
+
+
+def fa_debug_set_wait_limit_ns(ns: int) -> None:
+    """C ``fa_debug_set_wait_limit_ns`` (test hook): limit of every bounded wait; 0 restores 2 s."""
+    code = _abi.load().fa_debug_set_wait_limit_ns(int(ns))
+    if code != _abi.FA_OK:
+        raise FaError(code, "fa_debug_set_wait_limit_ns")
+
+
+def fa_debug_inject_stall(kernel_id: int) -> None:
+    """C ``fa_debug_inject_stall`` (test hook): CTA 0 of that kernel withholds its first P arrive; 0 = off."""
+    code = _abi.load().fa_debug_inject_stall(int(kernel_id))
+    if code != _abi.FA_OK:
+        raise FaError(code, "fa_debug_inject_stall")
 
 
 def fa_timing_enable(enable: bool = True) -> None:

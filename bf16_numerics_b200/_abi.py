@@ -27,12 +27,18 @@ FA_KERNEL_BWD_DELTA = 1
 FA_KERNEL_BWD_MAIN = 2
 FA_KERNEL_BWD_DQ = 3
 FA_NUM_KERNELS = 4
+
+# kernel ids in the device error word (fa_device_error) and for fa_debug_inject_stall
+FA_ERRWORD_FWD = 1
+FA_ERRWORD_BWD_D64 = 3
+FA_ERRWORD_BWD_D128 = 4
 KERNEL_NAMES = ("fa_fwd_kernel", "fa_bwd_delta_kernel", "fa_bwd_main_kernel", "fa_bwd_dq_convert_kernel")
 
 # every symbol include/fa_b200.h declares
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_workspace_delta_offset",
            "fa_bwd_workspace_dq_offset", "fa_status_string", "fa_device_error", "fa_timing_enable",
-           "fa_timing_read", "fa_bwd_noalloc", "fa_last_error_string", "fa_fwd_o_hp", "fa_bwd_o_hp")
+           "fa_timing_read", "fa_bwd_noalloc", "fa_last_error_string", "fa_fwd_o_hp", "fa_bwd_o_hp",
+           "fa_debug_set_wait_limit_ns", "fa_debug_inject_stall")
 
 
 class FaRowStats(ctypes.Structure):
@@ -68,6 +74,10 @@ def load() -> ctypes.CDLL:
     lib.fa_last_error_string.restype = ctypes.c_char_p
     lib.fa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.fa_device_error.restype = i
+    lib.fa_debug_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.fa_debug_set_wait_limit_ns.restype = i
+    lib.fa_debug_inject_stall.argtypes = [ctypes.c_uint]
+    lib.fa_debug_inject_stall.restype = i
     lib.fa_timing_enable.argtypes = [i]
     lib.fa_timing_enable.restype = i
     lib.fa_timing_read.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]

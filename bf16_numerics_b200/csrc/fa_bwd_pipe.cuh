@@ -144,7 +144,8 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   // per-query vectors at VEC_OFF, [stage][0]: -a, [stage][1]: 1/l, [stage][2]: delta (fp32 x 128)
-  const BoundedWait wait{abort_flag, 3u};
+  const uint64_t limit_ns = wait_limit_ns();
+  const BoundedWait wait{abort_flag, 3u, limit_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -193,7 +194,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     if (warp == 13) {
       tc_fence_after();
       volatile int never = 0;
-      const BoundedWait drain{&never, 3u};
+      const BoundedWait drain{&never, 3u, limit_ns};
       drain(bar(L::TEARDOWN), 0, 30);
       tmem_dealloc(tmem, L::TMEM_COLS);
     }
@@ -241,7 +242,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         g += cur.n;
       }
       volatile int never = 0;
-      const BoundedWait drain{&never, 3u};
+      const BoundedWait drain{&never, 3u, limit_ns};
       if (last_r >= 0) drain(bar(L::KV_FULL), last_r & 1, 20);
       for (int s = 0; s < NST; ++s)
         if (issued[s] >= 0) drain(bar(L::Q_FULL + s), (issued[s] / NST) & 1, 21);
@@ -471,6 +472,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     // warpgroups leave together and neither is left waiting on a barrier the
     // other no longer reaches.
     bool ok = true;
+    const bool stall = inject_stall_here(3u);  // test hook (fa_debug_inject_stall)
     for (; cur.valid; cur.next_item()) {
       bool leave = false;
       for (int i = 0; i < cur.n; ++i, ++g) {
@@ -531,7 +533,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (threadIdx.x == 0) FA_TRACE_POINT(27);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(L::P_FULL + b));
+        if (!(stall && g == 0)) mbar_arrive(bar(L::P_FULL + b));
         if (threadIdx.x == 0) FA_TRACE_POINT(21);
         ok = wait.warp(bar(L::DP_FULL), g & 1, 10);
         if (threadIdx.x == 0) FA_TRACE_POINT(22);

@@ -99,7 +99,8 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
   auto bar = [&](int i) { return base + L::BAR_OFF + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
-  const BoundedWait wait{abort_flag, 4u};
+  const uint64_t limit_ns = wait_limit_ns();
+  const BoundedWait wait{abort_flag, 4u, limit_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -141,7 +142,7 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
     if (warp == 13) {
       tc_fence_after();
       volatile int never = 0;
-      const BoundedWait drain{&never, 4u};
+      const BoundedWait drain{&never, 4u, limit_ns};
       drain(bar(L::TEARDOWN), 0, 30);
       tmem_dealloc(tmem, L::TMEM_COLS);
     }
@@ -193,7 +194,7 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
         g += cur.n;
       }
       volatile int never = 0;
-      const BoundedWait drain{&never, 4u};
+      const BoundedWait drain{&never, 4u, limit_ns};
       if (last_r >= 0) drain(bar(L::KV_FULL), last_r & 1, 20);
       for (int s = 0; s < NST; ++s)
         if (issued[s] >= 0) drain(bar(L::Q_FULL + s), (issued[s] / NST) & 1, 21);
@@ -403,6 +404,7 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
     // named barrier 1 once per block (an AND vote); a bounded wait that gives
     // up only clears `ok`, and the next vote takes both warpgroups out.
     bool ok = true;
+    const bool stall = inject_stall_here(4u);  // test hook (fa_debug_inject_stall)
     for (; cur.valid; cur.next_item()) {
       bool leave = false;
       for (int i = 0; i < cur.n; ++i, ++g) {
@@ -475,7 +477,7 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
         tmem_st32(tmem + lane_base + L::S_COL + 32u * h, pk);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(L::P_FULL));
+        if (!(stall && g == 0)) mbar_arrive(bar(L::P_FULL));
         ok = wait.warp(bar(L::DP_FULL), g & 1, 10);
         if (!ok) continue;  // the next meeting takes everyone out
         tc_fence_after();

@@ -147,7 +147,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   auto bar = [&](int i) { return base + L::BAR_OFF + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
-  const BoundedWait wait{abort_flag, 1u};
+  const uint64_t limit_ns = wait_limit_ns();
+  const BoundedWait wait{abort_flag, 1u, limit_ns};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -193,7 +194,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (warp == 9) {
       tc_fence_after();
       volatile int never = 0;
-      const BoundedWait drain{&never, 1u};
+      const BoundedWait drain{&never, 1u, limit_ns};
       drain(bar(L::TEARDOWN), 0, 30);  // every MMA of this CTA has completed
       tmem_dealloc(tmem, L::TMEM_COLS);
     }
@@ -275,7 +276,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // drain: every load issued must have landed before the CTA may exit
       // (the last two uses of each two-slot ring)
       volatile int never = 0;
-      const BoundedWait drain{&never, 1u};
+      const BoundedWait drain{&never, 1u, limit_ns};
       for (int g = q_issued - 2; g < q_issued; ++g)
         if (g >= 0) drain(bar(L::Q_FULL + (g & 1)), (g >> 1) & 1, 20);
       for (int g = k_issued - 2; g < k_issued; ++g)
@@ -374,6 +375,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // together and neither is left waiting on a barrier the other no longer
     // reaches.
     bool ok = true;
+    const bool stall = inject_stall_here(1u);  // test hook (fa_debug_inject_stall)
     FwdCursor cur;
     cur.start(p);
     int gt = 0;
@@ -541,7 +543,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         l += psum;
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(L::P_FULL));
+        if (!(stall && gt == 0)) mbar_arrive(bar(L::P_FULL));
         if (threadIdx.x == 0) FA_TRACE_POINT(24);
       }
       if (left) break;

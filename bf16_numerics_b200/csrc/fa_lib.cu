@@ -248,9 +248,12 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   return e == cudaSuccess ? FA_OK : cuda_fail("fa_fwd_kernel launch", e);
 }
 
+// Grid of a memory-bound kernel: one block per `per_block` units of work,
+// at most 16 resident 256-thread blocks per SM (grid-stride loops take the rest).
 int grid_for(long long work, int per_block) {
   long long g = (work + per_block - 1) / per_block;
-  if (g > 148 * 16) g = 148 * 16;
+  const long long cap = 16ll * (sm_count() > 0 ? sm_count() : 148);
+  if (g > cap) g = cap;
   if (g < 1) g = 1;
   return static_cast<int>(g);
 }
@@ -327,8 +330,6 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       if (e == cudaSuccess) e = cudaGetLastError();
       if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
     }
-    const cudaError_t e = cudaSuccess;
-    if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
   }
   {
     const long long n8 = rows * D / 8;
@@ -478,6 +479,22 @@ fa_status fa_device_error(unsigned int* code) {
     if (cudaMemcpyToSymbol(fa::g_fa_error, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
     return FA_ERR_TIMEOUT;
   }
+  return FA_OK;
+}
+
+fa_status fa_debug_set_wait_limit_ns(unsigned long long ns) {
+  const unsigned long long v = ns == 0 ? 2000000000ull : ns;
+  if (cudaMemcpyToSymbol(fa::g_fa_wait_limit_ns, &v, sizeof(v)) != cudaSuccess)
+    return cuda_fail("cudaMemcpyToSymbol(wait limit)", cudaGetLastError());
+  return FA_OK;
+}
+
+fa_status fa_debug_inject_stall(unsigned int kernel_id) {
+  if (kernel_id != 0 && kernel_id != FA_ERRWORD_FWD && kernel_id != FA_ERRWORD_BWD_D64 &&
+      kernel_id != FA_ERRWORD_BWD_D128)
+    return FA_ERR_INVALID_ARG;
+  if (cudaMemcpyToSymbol(fa::g_fa_inject, &kernel_id, sizeof(kernel_id)) != cudaSuccess)
+    return cuda_fail("cudaMemcpyToSymbol(stall injection)", cudaGetLastError());
   return FA_OK;
 }
 

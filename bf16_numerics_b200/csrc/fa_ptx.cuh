@@ -71,11 +71,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Code layout: kernel id << 24 | wait site << 16 | low 16 bits of blockIdx.x.
 __device__ unsigned int g_fa_error = 0;
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+// Time limit of every bounded wait (2 s by default: far above any legitimate
+// wait).  A test may lower it (fa_debug_set_wait_limit_ns) to exercise the
+// exit path quickly.
+__device__ unsigned long long g_fa_wait_limit_ns = 2000000000ull;
+
+// Test hook (fa_debug_inject_stall): when it equals a kernel's id, CTA 0 of
+// that kernel withholds the first arrive of its elementwise warps on the
+// barrier that hands P_bar (forward) or P^T (backward) to the MMA warp.  The
+// MMA warp's bounded wait then runs out with no bulk copy outstanding on that
+// barrier, and the kernel takes its error exit.  0: no injection.
+__device__ unsigned int g_fa_inject = 0;
+
+__device__ __forceinline__ uint64_t wait_limit_ns() { return g_fa_wait_limit_ns; }
+__device__ __forceinline__ bool inject_stall_here(uint32_t kernel_id) {
+  return blockIdx.x == 0 && g_fa_inject == kernel_id;
+}
 
 struct BoundedWait {
   volatile int* abort_flag;  // in shared memory, one per CTA
   uint32_t kernel_id;
+  uint64_t limit_ns;
 
   // Returns true when the phase with the given parity has completed; false if
   // the CTA is aborting (this wait timed out, or another one did).
@@ -86,7 +102,7 @@ struct BoundedWait {
       if (mbar_try_wait(bar, parity)) return true;
       if ((it & 255u) == 0u) {
         if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
           atomicCAS(&g_fa_error, 0u, (kernel_id << 24) | ((site & 0xFFu) << 16) | (blockIdx.x & 0xFFFFu));
           *abort_flag = 1;
           __threadfence_block();
@@ -329,11 +345,14 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 // Functions", 1980): y = k + r with k = round(y) taken by adding and removing
 // 1.5 * 2^23, r in [-1/2, 1/2] exact; 2^r by a degree-5 polynomial with
 // constant term 1, fitted for this library by relative least squares with
-// Lawson reweighting on [-1/2, 1/2] (max relative error 1.9e-7 in fp32
-// Horner form, the accuracy class of ex2.approx); 2^k by adding k to the
+// Lawson reweighting on [-1/2, 1/2] (20001 equispaced points, 300 solves;
+// the fit is re-run by the CPU test of this function; max relative error
+// 1.1e-7 with the fp32-rounded coefficients in exact arithmetic, 1.9e-7 in
+// fp32 Horner form, the accuracy class of ex2.approx); 2^k by adding k to the
 // exponent field.  y = 0 gives exactly 1.  Arguments below -126 (masked
-// scores are -inf) are clamped to -126: the result is then 2^-126 instead of
-// 0, far below anything that reaches a bf16 operand or the fp32 row sum.
+// scores are -inf) give exactly 0, as ex2.approx.ftz does: the range
+// reduction works on the argument clamped to -126 and the result is replaced
+// by 0 afterwards, so a masked key never enters the row sum or P_bar V.
 __device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t y) {
   float y0, y1;
   f2_unpack(y, y0, y1);
@@ -341,9 +360,9 @@ __device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t y) {
   const uint64_t kMagic = f2_pack(12582912.f, 12582912.f);  // 1.5 * 2^23
   const uint64_t t = f2_add(yc, kMagic);                     // 1.5 * 2^23 + k
   const uint64_t r = f2_sub(yc, f2_sub(t, kMagic));          // y - k
-  uint64_t q = f2_fma(f2_pack(0.0013264636509120464f, 0.0013264636509120464f), r,
-                      f2_pack(0.009671482257544994f, 0.009671482257544994f));
-  q = f2_fma(q, r, f2_pack(0.05550733581185341f, 0.05550733581185341f));
+  uint64_t q = f2_fma(f2_pack(0.0013264708686619997f, 0.0013264708686619997f), r,
+                      f2_pack(0.009671511128544807f, 0.009671511128544807f));
+  q = f2_fma(q, r, f2_pack(0.05550733953714371f, 0.05550733953714371f));
   q = f2_fma(q, r, f2_pack(0.24022242426872253f, 0.24022242426872253f));
   q = f2_fma(q, r, f2_pack(0.6931470036506653f, 0.6931470036506653f));
   q = f2_fma(q, r, f2_pack(1.f, 1.f));
@@ -352,8 +371,9 @@ __device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t y) {
   f2_unpack(t, t0, t1);
   // the low bits of t hold k (two's complement): shifting them to the
   // exponent field drops the 1.5 * 2^23 part
-  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+  const float e0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  const float e1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+  return f2_pack(y0 < -126.f ? 0.f : e0, y1 < -126.f ? 0.f : e1);
 }
 }  // namespace fa
 

@@ -150,10 +150,33 @@ const char* fa_last_error_string(void);
 
 /* Synchronises the current device, then reads and clears the device error
  * word that kernels set when a bounded wait ran out.  *code (may be NULL)
- * receives the raw word (kernel id << 24 | wait site << 16 | block).
- * Returns FA_OK if it was clear, FA_ERR_TIMEOUT if set, FA_ERR_CUDA if the
- * synchronisation failed. */
+ * receives the raw word (kernel id << 24 | wait site << 16 | block), the
+ * kernel id being one of FA_ERRWORD_*.  Returns FA_OK if it was clear,
+ * FA_ERR_TIMEOUT if set, FA_ERR_CUDA if the synchronisation failed. */
+enum { FA_ERRWORD_FWD = 1, FA_ERRWORD_BWD_D64 = 3, FA_ERRWORD_BWD_D128 = 4 };
 fa_status fa_device_error(unsigned int* code);
+
+/* Test hooks for the bounded-wait exit path (the pages have no counterpart;
+ * they exist so that the error exit can be exercised on a GPU without a
+ * fault).  Both write a device variable of the current device with a
+ * synchronous copy; call them between launches, never while a kernel of this
+ * library runs.
+ *
+ * fa_debug_set_wait_limit_ns: time limit of every bounded wait of every
+ * kernel launched afterwards (0 restores the default, 2 s).  A short limit
+ * (milliseconds) makes a withheld arrive end quickly; it must stay well above
+ * the longest legitimate wait of the problem being run.
+ *
+ * fa_debug_inject_stall: kernel_id = FA_ERRWORD_FWD, _BWD_D64 or _BWD_D128
+ * makes CTA 0 of every later launch of that kernel withhold its elementwise
+ * warps' first arrive on the barrier that hands P_bar (forward) or P^T
+ * (backward) to the MMA warp.  No bulk copy is outstanding on that barrier:
+ * the MMA warp's wait runs out, the kernel records the error word, drains its
+ * copies and products, frees its tensor memory and returns; fa_device_error
+ * then reports FA_ERR_TIMEOUT, and the outputs of that launch are undefined.
+ * 0 switches the injection off.  Any other id: FA_ERR_INVALID_ARG. */
+fa_status fa_debug_set_wait_limit_ns(unsigned long long ns);
+fa_status fa_debug_inject_stall(unsigned int kernel_id);
 
 /* Per-kernel timing.  While enabled, every launch made by fa_fwd / fa_bwd is
  * bracketed by two CUDA events recorded on the launching stream.
@@ -186,7 +209,10 @@ fa_status fa_timing_read(int* launches, double* total_ms);
  * the last call's contents (the dQ accumulator is cleared by the call itself
  * before use), so calls that overlap on the GPU -- on different streams, or
  * from different host threads -- race on it and must be serialised by the
- * caller.  Returns FA_ERR_CUDA if the address lookup fails. */
+ * caller.  The looked-up address is kept for the life of the process: a
+ * device reset (cudaDeviceReset) or any other teardown of the device's
+ * primary context invalidates it, and calling fa_bwd_noalloc after one is not
+ * supported.  Returns FA_ERR_CUDA if the address lookup fails. */
 #define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const float* lse, const float* row_m, void* dq, void* dk, void* dv, int B, int H, int N,

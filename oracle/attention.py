@@ -52,6 +52,8 @@ from __future__ import annotations
 
 import numpy as np
 
+from .bf16 import round_bf16
+
 STANDARD = 0
 STABILIZED = 1
 STABILIZED_MARGIN = 2
@@ -159,12 +161,16 @@ def attention_fwd(q, k, v, causal: bool = True, mode: int = STABILIZED, beta: fl
 
 
 def attention_bwd(q, k, v, do, causal: bool = True, mode: int = STABILIZED, beta: float = 2.0,
-                  fwd: dict | None = None, o_for_delta=None) -> dict:
+                  fwd: dict | None = None, o_for_delta=None, ds_bf16: bool = False) -> dict:
     """Backward pass: float64 dq, dk, dv [B,H,N,d] and delta [B,H,N].
 
     ``fwd`` is this module's forward result (recomputed if None).  delta uses
     the oracle's own O unless ``o_for_delta`` (e.g. a BF16 O from elsewhere)
-    is given.
+    is given.  ``ds_bf16`` models the BF16 operand of the dQ and dK products
+    (the pages' training runs in BF16, page 1 "mechanism two"): dS is rounded
+    to the nearest BF16 value (through binary32, RNE, by the emulator in
+    oracle.bf16) before dQ = dS K * scale and dK = dS^T Q * scale; every other
+    step stays float64.
     """
     q, k, v, do = (_split_heads(x) for x in (q, k, v, do))
     if fwd is None:
@@ -191,6 +197,8 @@ def attention_bwd(q, k, v, do, causal: bool = True, mode: int = STABILIZED, beta
             dv[b, h] = p.T @ dob
             dp = dob @ v[b, h].astype(np.float64).T
             ds = p * (dp - dlt[:, None])
+            if ds_bf16:
+                ds = round_bf16(ds.astype(np.float32)).astype(np.float64)
             dq[b, h] = ds @ k[b, h].astype(np.float64) * sc
             dk[b, h] = ds.T @ q[b, h].astype(np.float64) * sc
             delta[b, h] = dlt

@@ -150,3 +150,10 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "libfa_b200.so"))
     with pytest.raises(ImportError):
         _abi.load()
+
+
+def test_inject_stall_rejects_unknown_kernel_ids_before_touching_cuda(lib):
+    # only the error-word ids of the three kernels with bounded waits (and 0) are accepted
+    for bad in (2, 5, 255, 1 << 24):
+        assert lib.fa_debug_inject_stall(bad) == _abi.FA_ERR_INVALID_ARG
+    assert (_abi.FA_ERRWORD_FWD, _abi.FA_ERRWORD_BWD_D64, _abi.FA_ERRWORD_BWD_D128) == (1, 3, 4)

@@ -10,20 +10,20 @@ def test_traffic_record_is_keyed_by_kernel_workload_and_sources(tmp_path, monkey
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "traffic.txt").write_text(
         "# kernel workload source_hash unit bytes\n"
-        "fa_bwd_main_kernel g2s abc123 bytes 1000\n"
-        "fa_bwd_main_kernel long abc123 bytes 5000\n"
-        "fa_fwd_kernel g2s oldhash bytes 7\n")
+        "fa_bwd_main_pipe_kernel g2s abc123 bytes 1000\n"
+        "fa_bwd_main_pipe128_kernel long abc123 bytes 5000\n"
+        "fa_fwd_kernel<64> g2s oldhash bytes 7\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc123")
-    assert bench.recorded_traffic("fa_bwd_main_kernel", "g2s") == 1000.0
-    assert bench.recorded_traffic("fa_bwd_main_kernel", "long") == 5000.0
-    assert bench.recorded_traffic("fa_bwd_main_kernel", "tiestress") is None  # no capture for it
-    assert bench.recorded_traffic("fa_fwd_kernel", "g2s") is None  # taken on other sources
+    assert bench.recorded_traffic("fa_bwd_main_pipe_kernel", "g2s") == 1000.0
+    assert bench.recorded_traffic("fa_bwd_main_pipe128_kernel", "long") == 5000.0
+    assert bench.recorded_traffic("fa_bwd_main_pipe_kernel", "tiestress") is None  # no capture for it
+    assert bench.recorded_traffic("fa_fwd_kernel<64>", "g2s") is None  # taken on other sources
 
 
 def test_traffic_record_missing_file(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.recorded_traffic("fa_bwd_main_kernel", "g2s") is None
+    assert bench.recorded_traffic("fa_bwd_main_pipe_kernel", "g2s") is None
 
 
 def test_committed_traffic_lines_parse():
@@ -79,3 +79,12 @@ def test_peaks_fall_back_when_the_file_is_missing(tmp_path, monkeypatch):
     peaks, src = bench.load_peaks()
     assert src == "fallback"
     assert peaks == bench.FALLBACK_PEAKS
+
+
+def test_launched_kernel_names_follow_the_head_dimension():
+    import bench
+
+    assert bench.launched_kernel_name("fa_bwd_main_kernel", 64) == "fa_bwd_main_pipe_kernel"
+    assert bench.launched_kernel_name("fa_bwd_main_kernel", 128) == "fa_bwd_main_pipe128_kernel"
+    assert bench.launched_kernel_name("fa_fwd_kernel", 128) == "fa_fwd_kernel<128>"
+    assert bench.launched_kernel_name("fa_bwd_delta_kernel", 64) == "fa_bwd_delta_kernel"

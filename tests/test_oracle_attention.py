@@ -354,28 +354,35 @@ def test_planted_mistake_swapped_branch_is_caught(monkeypatch):
         check_shift_rule(swapped)
 
 
+def _oracle_bwd_with(monkeypatch, old: str, new: str):
+    """Replace one expression in the source of oracle.attention.attention_bwd
+    and install the result in the oracle module (undone by monkeypatch)."""
+    import inspect
+    import textwrap
+
+    src = textwrap.dedent(inspect.getsource(A.attention_bwd))
+    assert src.count(old) == 1, old
+    ns = dict(vars(A))
+    exec(compile(src.replace(old, new), A.__file__, "exec"), ns)
+    monkeypatch.setattr(A, "attention_bwd", ns["attention_bwd"])
+
+
 def test_planted_mistake_transposed_dk_is_caught(monkeypatch):
-    rng = np.random.default_rng(11)
-    q, k, v, do = (_rand_bf16(rng, (1, 1, 16, 16)) for _ in range(4))
-    good = A.attention_bwd(q, k, v, do, True, 1)
-    _, _, dk, _ = _torch_ref(q, k, v, do, True)
-    np.testing.assert_allclose(good["dk"], dk, rtol=1e-9, atol=1e-11)
-    # the slip: dK = dS Q instead of dS^T Q, i.e. a transposed operand
-    real_matmul = np.matmul
+    """The slip planted in the oracle itself: dK = dS Q instead of dS^T Q (a
+    transposed operand; square shapes keep it well-formed).  The torch SDPA
+    pin rejects it."""
+    _oracle_bwd_with(monkeypatch, "ds.T @ q[b, h]", "ds @ q[b, h]")
+    with pytest.raises(AssertionError):
+        test_against_torch_sdpa_float64(True, 1)
+    with pytest.raises(AssertionError):
+        test_gradients_finite_differences(False, 1)
 
-    class Slip:
-        @staticmethod
-        def run():
-            s = q[0, 0].astype(np.float64) @ k[0, 0].astype(np.float64).T / 4.0
-            s = np.where(np.tril(np.ones((16, 16), bool)), s, -np.inf)
-            p = np.exp(s - s.max(1, keepdims=True))
-            p /= p.sum(1, keepdims=True)
-            dp = do[0, 0].astype(np.float64) @ v[0, 0].astype(np.float64).T
-            o = p @ v[0, 0].astype(np.float64)
-            ds = p * (dp - (do[0, 0] * o).sum(1, keepdims=True))
-            return real_matmul(ds, q[0, 0].astype(np.float64)) / 4.0
 
-    assert not np.allclose(Slip.run(), dk[0, 0], rtol=1e-6)
+def test_planted_mistake_dq_without_scale_is_caught(monkeypatch):
+    """The slip planted in the oracle itself: dQ without the softmax scale."""
+    _oracle_bwd_with(monkeypatch, "ds @ k[b, h].astype(np.float64) * sc", "ds @ k[b, h].astype(np.float64)")
+    with pytest.raises(AssertionError):
+        test_against_torch_sdpa_head_dims(64)
 
 
 def test_planted_mistake_dropped_delta_is_caught():
@@ -424,3 +431,73 @@ def test_planted_mistake_tie_count_of_one_is_caught(monkeypatch):
     assert tied.any()
     assert np.all(f["pbar"].max(axis=-1)[tied] == 1.0)  # the fix's pin (max P_bar < 1) fails
 
+
+
+# ------------------------------------- BF16 dS operand (rounding point of dQ, dK)
+
+def _brute_bwd_bf16_ds(q, k, v, do, causal):
+    """dQ, dK with dS rounded to BF16 before the two products, written with
+    pure-Python loops; the rounding is torch's float32 -> bfloat16 cast (an
+    implementation independent of oracle.bf16)."""
+    N, d = q.shape
+    sc = 1.0 / math.sqrt(d)
+    vis = [[(j <= i) if causal else True for j in range(N)] for i in range(N)]
+    s = [[sum(float(q[i, c]) * float(k[j, c]) for c in range(d)) * sc for j in range(N)] for i in range(N)]
+    p = [[0.0] * N for _ in range(N)]
+    for i in range(N):
+        z = sum(math.exp(s[i][j]) for j in range(N) if vis[i][j])
+        for j in range(N):
+            p[i][j] = math.exp(s[i][j]) / z if vis[i][j] else 0.0
+    o = [[sum(p[i][j] * float(v[j, c]) for j in range(N)) for c in range(d)] for i in range(N)]
+    dlt = [sum(float(do[i, c]) * o[i][c] for c in range(d)) for i in range(N)]
+    ds = [[p[i][j] * (sum(float(do[i, c]) * float(v[j, c]) for c in range(d)) - dlt[i]) for j in range(N)]
+          for i in range(N)]
+    dsb = torch.tensor(ds, dtype=torch.float64).to(torch.float32).to(torch.bfloat16).to(torch.float64).tolist()
+    dq = [[sum(dsb[i][j] * float(k[j, c]) for j in range(N)) * sc for c in range(d)] for i in range(N)]
+    dk = [[sum(dsb[i][j] * float(q[i, c]) for i in range(N)) * sc for c in range(d)] for j in range(N)]
+    return np.array(dq), np.array(dk), np.array(ds)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_bf16_ds_operand_brute_force(causal):
+    rng = np.random.default_rng(17)
+    N, d = 7, 8
+    q, k, v, do = (_rand_bf16(rng, (1, 1, N, d)) for _ in range(4))
+    k[0, 0, 4] = k[0, 0, 1]
+    q[0, 0, 5] = k[0, 0, 1]
+    f = A.attention_fwd(q, k, v, causal, 1)
+    b = A.attention_bwd(q, k, v, do, causal, 1, fwd=f, ds_bf16=True)
+    dq, dk, ds = _brute_bwd_bf16_ds(q[0, 0], k[0, 0], v[0, 0], do[0, 0], causal)
+    np.testing.assert_allclose(b["dq"][0, 0], dq, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(b["dk"][0, 0], dk, rtol=1e-12, atol=1e-13)
+    # dV and delta do not go through the rounded operand
+    b0 = A.attention_bwd(q, k, v, do, causal, 1, fwd=f)
+    assert np.array_equal(b["dv"], b0["dv"]) and np.array_equal(b["delta"], b0["delta"])
+    # the rounding moved dQ, and by no more than its a-priori bound
+    # |bf16(x) - x| <= 2^-8 |x|, summed over the product: 2^-8 * scale * |dS| |K|
+    bound = 2.0 ** -8 / math.sqrt(d) * (np.abs(ds) @ np.abs(k[0, 0].astype(np.float64)))
+    diff = np.abs(b["dq"][0, 0] - b0["dq"][0, 0])
+    assert diff.max() > 0 and np.all(diff <= bound * (1 + 1e-9) + 1e-300)
+
+
+def test_bf16_ds_floor_exceeds_the_float_bar_on_two_hot_rows():
+    """Why the reading is needed: where a row's softmax mass sits on two
+    bitwise-equal keys, dQ of that row is the small difference of two large,
+    nearly opposite dS terms times the same key, and the BF16 rounding of dS
+    alone moves it by more than 1e-2 of max|dQ| -- an exact product of
+    BF16-rounded dS cannot meet the float bar on such inputs, whatever the
+    kernel."""
+    # two existence cases (seed, N, query = s * key 0); over 36 such draws
+    # (three seeds, N in {64, 128, 200, 384}, s in {0.5, 0.75, 1}) the floor
+    # ranged from 0.17 % to 1.9 % of max|dQ|
+    errs = []
+    for seed, N, s in ((2, 200, 0.75), (31, 384, 1.0)):
+        rng = np.random.default_rng(seed)
+        q, k, v, do = (_rand_bf16(rng, (1, 1, N, 128)) for _ in range(4))
+        k[0, 0, N // 2] = k[0, 0, 0]
+        q[0, 0, N - 8:] = k[0, 0, 0] * np.float32(s)
+        f = A.attention_fwd(q, k, v, False, 1)
+        exact = A.attention_bwd(q, k, v, do, False, 1, fwd=f)
+        rounded = A.attention_bwd(q, k, v, do, False, 1, fwd=f, ds_bf16=True)
+        errs.append(np.abs(rounded["dq"] - exact["dq"]).max() / np.abs(exact["dq"]).max())
+    assert min(errs) > 1e-2, errs
