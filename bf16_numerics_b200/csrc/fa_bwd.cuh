@@ -23,7 +23,8 @@
 //   S^T  = K  Q_i^T   (A: K  smem K-major, B: Q_i  smem K-major)
 //   dP^T = V  dO_i^T  (A: V  smem K-major, B: dO_i smem K-major)
 //   dV  += P^T  dO_i  (A: P^T  TMEM,     B: dO_i smem MN-major, N = d)
-//   dK  += dS^T Q_i   (A: dS^T TMEM,     B: Q_i  smem MN-major, N = d)
+//   dK  += dS^T Q_i   (A: dS^T from TMEM (d = 128) or from the shared-memory
+//                      dS tile read K-major (d = 64), B: Q_i smem MN-major, N = d)
 //   dQ_i = dS   K     (A: dS smem MN-major (written from dS^T), B: K MN-major)
 #pragma once
 
@@ -33,7 +34,7 @@ namespace fa {
 
 // ------------------------------------------------------------------ delta
 // delta[r] = sum_c dO[r,c] * O[r,c] in fp32; also clears the dQ accumulator
-// row.  O is the bf16 output of the forward, or (OT = float) its fp32 value
+// (with TMA bulk stores of a zeroed shared-memory buffer).  O is the bf16 output of the forward, or (OT = float) its fp32 value
 // before rounding (the high-precision O_hp of the pages).
 // Memory bound: each row of O and dO is read once with 16-byte loads, LPR
 // lanes per row (8 elements of dO per lane); every warp takes U row groups at
@@ -93,12 +94,31 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
   constexpr int LPR = D / 8;               // lanes per row (8 elements per lane)
   constexpr int RPW = 32 / LPR;            // rows per warp per group
   constexpr int U = 4;                     // row groups per warp per pass
+  constexpr int ZCHUNK = 16384;            // bytes of zeros per bulk store
+  // zeros for the accumulator clear, written by TMA bulk stores so that the
+  // threads' own load/store slots stay with the delta rows
+  __shared__ __align__(128) float4 zeros[ZCHUNK / 16];
   const int lane = threadIdx.x & 31;
   const long long warp_global = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const int sub = lane / LPR, li = lane % LPR;
+  for (int i = threadIdx.x; i < ZCHUNK / 16; i += blockDim.x) zeros[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  fence_proxy_async_smem();
+  __syncthreads();
   grid_launch_dependents();
-  grid_dependency_wait();  // O comes from the forward grid
+  grid_dependency_wait();  // O comes from the forward grid; the workspace may be the previous grid's
+  if (threadIdx.x == 0) {
+    // this block's share of the fp32 dQ accumulator (rows * D * 4 bytes, a
+    // multiple of 256): 16 KB chunks dealt round-robin over the blocks
+    const long long bytes = rows * D * 4;
+    const long long nchunk = (bytes + ZCHUNK - 1) / ZCHUNK;
+    for (long long c = blockIdx.x; c < nchunk; c += gridDim.x) {
+      const long long off = c * ZCHUNK;
+      const long long len = bytes - off < ZCHUNK ? bytes - off : ZCHUNK;
+      bulk_store(reinterpret_cast<uint8_t*>(dq_acc) + off, smem_u32(zeros), static_cast<uint32_t>(len));
+    }
+    bulk_commit();
+  }
   for (long long r0 = warp_global * (RPW * U); r0 < rows; r0 += n_warps * (RPW * U)) {
     ORaw<OT> a[U];
     uint4 b[U];
@@ -115,15 +135,6 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const long long r = r0 + u * RPW + sub;
-      if (r < rows) {
-        float4* z = reinterpret_cast<float4*>(dq_acc + r * D) + 2 * li;
-        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
       float acc = a[u].dot(b[u], 0.f);
 #pragma unroll
       for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -131,6 +142,8 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
       if (r < rows && li == 0) delta[r] = acc;
     }
   }
+  // the zeros must stay in shared memory until the bulk stores are complete
+  if (threadIdx.x == 0) bulk_wait_all();
 }
 
 // --------------------------------------------------------------- dQ convert

@@ -16,11 +16,14 @@
 //     a key row: warpgroup h takes columns [64h, 64h+64).  Both copy their S^T
 //     columns to registers and meet at a named barrier; then warpgroup h
 //     writes its bf16 P^T into S^T cols [32h, 32h+32), so P^T occupies
-//     [0,64) and [64,128) is free for dQ.  dS^T goes into the first half of
-//     the dP^T columns each warpgroup has just read (64h + [0,32)), which
-//     needs no barrier.
-//   * dQ_g = dS K is one N = 64 product into S^T cols [64,128) of the same
-//     buffer, which no later product of the block touches.
+//     [0,64) and [64,128) is free for dQ.  Once they hold dP^T in registers
+//     they release its columns, so dP^T of the next block is computed while
+//     they form dS.
+//   * dS goes to shared memory only: a double-buffered [keys][queries] bf16
+//     tile (128B-swizzled, two 64-query halves) that is the A operand of both
+//     dK += dS^T Q (read K-major) and dQ_g = dS K (read MN-major).  dQ_g is
+//     one N = 64 product into S^T cols [64,128) of the block's S^T buffer,
+//     which no later product of the block touches.
 //   * Four drain warps move the dQ partial from TMEM into a 128B-swizzled
 //     fp32 staging box in shared memory and add it to the fp32 accumulator in
 //     global memory with one TMA tensor reduce-add per 32-column half, one
@@ -50,8 +53,8 @@ struct BwdPipeLayout {
   static constexpr int D = 64, B = 128, TILE = 128 * 64 * 2, NST = 3;
   static constexpr int K_OFF = 0, V_OFF = TILE, Q_OFF = 2 * TILE;
   static constexpr int DO_OFF = Q_OFF + NST * TILE;
-  static constexpr int DS_OFF = DO_OFF + NST * TILE;  // dS^T [keys][queries], two 64-query halves
-  static constexpr int DQS_OFF = DS_OFF + 2 * TILE;   // dQ staging: one [128 rows][32 fp32] swizzled box
+  static constexpr int DS_OFF = DO_OFF + NST * TILE;  // [2 buffers] dS^T [keys][queries], two 64-query halves
+  static constexpr int DQS_OFF = DS_OFF + 4 * TILE;   // dQ staging: one [128 rows][32 fp32] swizzled box
   static constexpr int VEC_OFF = DQS_OFF + TILE;      // [2 stages][3][128] fp32
   static constexpr int BAR_OFF = VEC_OFF + 2 * 3 * 128 * 4;
   enum {
@@ -62,6 +65,7 @@ struct BwdPipeLayout {
     S_FULL = Q_EMPTY + NST,    // [2]
     P_FULL = S_FULL + 2,       // [2]
     DP_FULL = P_FULL + 2,
+    DP_FREE,                   // the elementwise warps hold dP^T of the block in registers
     DS_FULL,
     DQ_FULL,                   // [2]
     DQ_FREE = DQ_FULL + 2,
@@ -78,6 +82,7 @@ struct BwdPipeLayout {
   static constexpr int THREADS = 512;
   static constexpr uint32_t REGS_ELEM = 168, REGS_DRAIN = 88, REGS_CTRL = 88;
 };
+static_assert(BwdPipeLayout::SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int x, int y, int z) {
   asm volatile(
@@ -164,6 +169,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       mbar_init(bar(L::VEC_EMPTY + b), 256);
     }
     mbar_init(bar(L::DP_FULL), 1);
+    mbar_init(bar(L::DP_FREE), 256);
     mbar_init(bar(L::DS_FULL), 256);
     mbar_init(bar(L::DQ_FREE), 128);
     mbar_init(bar(L::ACC_DONE), 1);
@@ -280,6 +286,9 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (!wait(bar(L::Q_FULL + (g0 % NST)), (g0 / NST) & 1, 3)) break;
         tc_fence_after();
         issue_s(g0);
+        // dP^T of the previous block has been copied to registers
+        if (g0 > 0 && !wait(bar(L::DP_FREE), (g0 - 1) & 1, 10)) break;
+        tc_fence_after();
         issue_dp(g0);
         if (n > 1) {
           if (!wait(bar(L::Q_FULL + ((g0 + 1) % NST)), ((g0 + 1) / NST) & 1, 3)) break;
@@ -299,26 +308,30 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           for (int ks = 0; ks < 8; ++ks)
             mma_ts(tmem + L::DV_COL, tmem + 128u * b + 8u * ks, sdesc_sw128(do_tile(g) + ks * 2048, 16384, 1024),
                    IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
+          // dP^T of the next block as soon as this block's dP^T is in registers
+          // (its Q/dO stage was waited for when S^T of that block was issued)
+          if (i + 1 < n) {
+            if (!wait(bar(L::DP_FREE), g & 1, 10)) { ok = false; break; }
+            tc_fence_after();
+            issue_dp(g + 1);
+          }
           if (!wait(bar(L::DS_FULL), g & 1, 5)) { ok = false; break; }
           FA_TRACE_POINT(11);
           tc_fence_after();
-          // dK += dS^T Q_g
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t a = tmem + L::DPT_COL + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4));
-            mma_ts(tmem + L::DK_COL, a, sdesc_sw128(q_tile(g) + ks * 2048, 16384, 1024), IDESC_KV,
-                   (i > 0 || ks > 0) ? 1u : 0u);
-          }
-          // dQ_g = dS K into S^T cols [64,128) of the same buffer
+          const uint32_t ds_tile = base + L::DS_OFF + 2 * b * TILE;
+          // dK += dS^T Q_g   (A: dS^T [keys][queries] in shared memory, K-major)
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + 128u * b + 64u, sdesc_sw128(base + L::DS_OFF + ks * 2048, 16384, 1024),
+            mma_ss(tmem + L::DK_COL, sdesc_sw128(ds_tile + (ks >> 2) * TILE + (ks & 3) * 32, 16, 1024),
+                   sdesc_sw128(q_tile(g) + ks * 2048, 16384, 1024), IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
+          // dQ_g = dS K into S^T cols [64,128) of the same buffer (A: the same tile, MN-major)
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + 128u * b + 64u, sdesc_sw128(ds_tile + ks * 2048, TILE, 1024),
                    sdesc_sw128(base + L::K_OFF + ks * 2048, 16384, 1024), IDESC_DQ, ks > 0 ? 1u : 0u);
           tc_commit(bar(L::DQ_FULL + b));
           tc_commit(bar(L::Q_EMPTY + (g % NST)));
-          if (i + 1 < n) {
-            issue_dp(g + 1);
-          } else {
+          if (i + 1 == n) {
             tc_commit(bar(L::ACC_DONE));  // dV, dK of this item complete
             tc_commit(bar(L::KV_EMPTY));  // K, V of this item no longer read
           }
@@ -461,7 +474,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     const uint64_t C2 = f2_pack(c_log2, c_log2);
     const bool mode1 = p.mode == 1;
     const int qoff = 64 * h;
-    const uint32_t ds_row = base + L::DS_OFF + h * TILE + t * 128;
+
     BwdCursor cur;
     cur.start(p);
     int g = 0;
@@ -537,8 +550,6 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (threadIdx.x == 0) FA_TRACE_POINT(21);
         ok = wait.warp(bar(L::DP_FULL), g & 1, 10);
         if (threadIdx.x == 0) FA_TRACE_POINT(22);
-        // the dQ product of the previous block has finished reading the dS tile
-        ok = ok && (g == 0 || wait.warp(bar(L::DQ_FULL + ((g - 1) & 1)), ((g - 1) >> 1) & 1, 11));
         if (!ok) continue;  // the next meeting takes everyone out
         tc_fence_after();
         uint32_t dpr[64];
@@ -548,6 +559,9 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           tmem_ld32x2(tmem + lane_base + L::DPT_COL + 64u * h, tmem + lane_base + L::DPT_COL + 64u * h + 32u, d0,
                       d1);
         }
+        // the dP^T columns may take the next block's product
+        tc_fence_before();
+        mbar_arrive(bar(L::DP_FREE));
         uint32_t dk_[32];
 #pragma unroll
         for (int pi = 0; pi < 32; pi += 2) {
@@ -564,16 +578,19 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           dk_[pi] = pack_bf16x2(d0, d1);
           dk_[pi + 1] = pack_bf16x2(d2, d3);
         }
-        // dS^T into the dP^T columns this warpgroup has read: 64h + [0,32)
-        tmem_st32(tmem + lane_base + L::DPT_COL + 64u * h, dk_);
+        // dS buffer b was last read by the dK and dQ products of block g-2
+        const bool buf_free = g < 2 || wait.warp(bar(L::DQ_FULL + b), ((g - 2) >> 1) & 1, 11);
+        ok = ok && buf_free;
         // dS^T row t, queries 64h + [0,64) = the eight 16-byte chunks of the half tile's row
+        // (after a wait that gave up, skip the write; the next vote takes everyone out)
+        if (buf_free) {
+          const uint32_t ds_row = base + L::DS_OFF + (2 * b + h) * TILE + t * 128;
 #pragma unroll
-        for (int chunk = 0; chunk < 8; ++chunk)
-          sts128(ds_row + ((chunk ^ (t & 7)) << 4), dk_[4 * chunk], dk_[4 * chunk + 1], dk_[4 * chunk + 2],
-                 dk_[4 * chunk + 3]);
+          for (int chunk = 0; chunk < 8; ++chunk)
+            sts128(ds_row + ((chunk ^ (t & 7)) << 4), dk_[4 * chunk], dk_[4 * chunk + 1], dk_[4 * chunk + 2],
+                   dk_[4 * chunk + 3]);
+        }
         fence_proxy_async_smem();
-        tmem_st_wait();
-        tc_fence_before();
         mbar_arrive(bar(L::DS_FULL));
         mbar_arrive(bar(L::VEC_EMPTY + b));
         if (threadIdx.x == 0) FA_TRACE_POINT(24);

@@ -220,15 +220,15 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   p.mode = mode;
   p.beta = beta;
   p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
-  // persistent: CTAS_PER_SM CTAs per SM (at most one per work item)
+  // persistent: one CTA per SM (at most one per work item; an item is
+  // FwdLayout::NT Q tiles of one (batch, head))
   const int n_sm = sm_count();
   if (n_sm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)");
-  const long long items = static_cast<long long>(p.n_qblk) * BH;
-  auto launch = [&](auto kernel, int smem, int ctas_per_sm) {
-    const long long slots = static_cast<long long>(n_sm) * ctas_per_sm;
-    const unsigned grid = static_cast<unsigned>(items < slots ? items : slots);
+  auto launch = [&](auto kernel, int smem, int nt) {
+    const long long items = static_cast<long long>((p.n_qblk + nt - 1) / nt) * BH;
+    const unsigned grid = static_cast<unsigned>(items < n_sm ? items : n_sm);
     LaunchTimer tm(FA_KERNEL_FWD, stream);
-    const cudaError_t err = launch_pdl(kernel, dim3(grid), dim3(384), smem, stream, mq, mk, mv, mo, p);
+    const cudaError_t err = launch_pdl(kernel, dim3(grid), dim3(512), smem, stream, mq, mk, mv, mo, p);
     tm.done();
     return err;
   };
@@ -237,12 +237,12 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
     using L = fa::FwdLayout<D, false>;
     static std::atomic<uint64_t> attr{0};
     if (!ensure_smem(fa::fa_fwd_kernel<D, false>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
-    e = launch(fa::fa_fwd_kernel<D, false>, L::SMEM_BYTES, L::CTAS_PER_SM);
+    e = launch(fa::fa_fwd_kernel<D, false>, L::SMEM_BYTES, L::NT);
   } else {
     using L = fa::FwdLayout<D, true>;
     static std::atomic<uint64_t> attr{0};
     if (!ensure_smem(fa::fa_fwd_kernel<D, true>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
-    e = launch(fa::fa_fwd_kernel<D, true>, L::SMEM_BYTES, L::CTAS_PER_SM);
+    e = launch(fa::fa_fwd_kernel<D, true>, L::SMEM_BYTES, L::NT);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : cuda_fail("fa_fwd_kernel launch", e);
