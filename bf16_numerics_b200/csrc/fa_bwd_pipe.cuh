@@ -28,8 +28,11 @@
 //     fp32 staging box in shared memory and add it to the fp32 accumulator in
 //     global memory with one TMA tensor reduce-add per 32-column half, one
 //     half after the other through the same box (rows past N are clipped by
-//     the tensor map).  They also prepare the per-query
-//     vectors (lse or m, 1/l, delta) two blocks ahead.
+//     the tensor map).  Two blocks later, once those reduce-adds are
+//     complete, they count the contribution on the query block's counter;
+//     the CTA that completes a query block converts it to bf16 dQ.  They
+//     also prepare the per-query vectors (lse or m, 1/l, delta) two blocks
+//     ahead.
 //
 // Barrier phases count a global query-block index g that runs across the
 // CTA's items; every phase of every barrier is waited for in order and no
@@ -402,11 +405,50 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     for (int k = 0; k < 2 && pub.valid; ++k, ++g_pub, pub.next_block()) publish_vec(g_pub, pub, load_vec(pub));
     Vec3 nxt = load_vec(pub);
     if (t == 0) tma_prefetch_desc(&tm_dq);
+    // dQ conversion in this kernel: after a block's reduce-adds are complete
+    // (checked two blocks later, so the drain does not stall on them), thread
+    // 0 counts that contribution on the query block's counter; the CTA whose
+    // count completes the block (query block qb has qb+1 contributions when
+    // causal, n_blk otherwise) converts its 128 rows to bf16.  The decision
+    // is broadcast through two flag slots used alternately, so one barrier
+    // per block suffices.
+    volatile int* conv_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
+    int n_counted = 0;
+    auto count_and_convert = [&](int bh, int qb) {
+      if (t == 0) {
+        fence_proxy_async_global();  // the completed reduce-adds, before the count
+        __threadfence();
+        const unsigned expected = static_cast<unsigned>(p.causal ? qb + 1 : p.n_blk);
+        const unsigned old = atomicAdd(p.dq_cnt + static_cast<size_t>(bh) * p.n_blk + qb, 1u);
+        __threadfence();
+        conv_flag[n_counted & 1] = (old + 1 == expected) ? 1 : 0;
+      }
+      named_barrier_sync(2, 128);
+      const bool last = conv_flag[n_counted & 1] != 0;
+      ++n_counted;
+      const int q = qb * L::B + t;
+      if (last && q < p.N) {
+        const size_t ri = static_cast<size_t>(bh) * p.N + q;
+        const float4* src = reinterpret_cast<const float4*>(p.dq_acc + ri * L::D);
+        uint4* dst = reinterpret_cast<uint4*>(p.dq + ri * L::D);
+        float4 a[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) a[c] = __ldcg(src + c);  // L2: written by other CTAs' reduce-adds
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          dst[c] = make_uint4(pack_bf16x2(a[2 * c].x, a[2 * c].y), pack_bf16x2(a[2 * c].z, a[2 * c].w),
+                              pack_bf16x2(a[2 * c + 1].x, a[2 * c + 1].y),
+                              pack_bf16x2(a[2 * c + 1].z, a[2 * c + 1].w));
+      }
+    };
+    // (batch*head, query block) of the last two blocks not yet counted
+    int pend_bh[2] = {0, 0}, pend_qb[2] = {0, 0};
     // A bounded wait that gives up only clears `ok`; the warpgroup leaves the
     // loop together at the AND vote on named barrier 2 (a stale TMEM read
     // before it is in bounds and harmless).
-    bool ok = true;
-    for (int g = 0; cur.valid; ++g, cur.next_block()) {
+    bool ok = true, aborted = false;
+    int g = 0;
+    for (; cur.valid; ++g, cur.next_block()) {
       const int b = g & 1;
       {
         // every lane calls the warp-uniform wait (ok may differ per lane here)
@@ -420,7 +462,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       tc_fence_before();
       mbar_arrive(bar(L::DQ_FREE));
       if (t == 0) bulk_wait_read_all();  // the previous reduce has finished reading the staging tile
-      if (!named_barrier_and(2, 128, ok)) break;
+      if (!named_barrier_and(2, 128, ok)) { aborted = true; break; }
       // row t of the 32-column box, 16-byte chunk c stored at chunk c ^ (t & 7);
       // the two halves of the row go through the box one after the other
       const uint32_t row = base + L::DQS_OFF + t * 128;
@@ -446,6 +488,14 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         }
       }
       if (t == 0) FA_TRACE_POINT(31);
+      // block g-2's two reduce-add groups are complete once at most four
+      // (blocks g-1 and g) are pending
+      if (g >= 2) {
+        if (t == 0) bulk_wait_allow<4>();
+        count_and_convert(pend_bh[b], pend_qb[b]);
+      }
+      pend_bh[b] = cur.bh;
+      pend_qb[b] = cur.qblk();
       if (pub.valid) {
         // block g+2 reuses the vector stage of block g
         // (a wait that gives up skips the publish; the next vote ends the loop)
@@ -459,6 +509,11 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       }
     }
     if (t == 0) bulk_wait_all();
+    if (!aborted) {
+      // the last two blocks
+      if (g >= 2) count_and_convert(pend_bh[g & 1], pend_qb[g & 1]);
+      if (g >= 1) count_and_convert(pend_bh[(g - 1) & 1], pend_qb[(g - 1) & 1]);
+    }
     teardown();
     return;
   }

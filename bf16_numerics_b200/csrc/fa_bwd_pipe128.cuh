@@ -60,7 +60,13 @@ struct BwdPipe128Layout {
   static constexpr int DO_OFF = Q_OFF + NST * TILE;
   static constexpr int DS_OFF = DO_OFF + NST * TILE;     // dS^T [keys][queries], two 64-query halves
   static constexpr int VEC_OFF = DS_OFF + TILE;          // [3][128] fp32: exponent offset, 1/l, delta
-  static constexpr int BAR_OFF = VEC_OFF + 3 * 128 * 4;
+  static constexpr int RING_OFF = VEC_OFF + 3 * 128 * 4; // [RING] item numbers (-1: end of the list)
+  static constexpr int RING = 4;
+  // threads that read each ring slot: the MMA thread, the 128 drain threads
+  // and the 256 elementwise threads twice (their block cursor and the cursor
+  // that prefetches the per-query vectors two blocks ahead)
+  static constexpr int RING_READERS = 1 + 128 + 2 * 256;
+  static constexpr int BAR_OFF = RING_OFF + RING * 4;
   enum {
     KV_FULL = 0,
     KV_EMPTY,
@@ -76,7 +82,9 @@ struct BwdPipe128Layout {
     ACC_FREE,
     DSTILE_FREE,  // the drain's reduce-adds have read the dS tile
     TEARDOWN,
-    NBAR
+    ITEM_FULL,              // [RING] the producer has published the slot's item
+    ITEM_EMPTY = ITEM_FULL + 4,  // [RING] every reader has read it
+    NBAR = ITEM_EMPTY + 4
   };
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
@@ -85,6 +93,65 @@ struct BwdPipe128Layout {
   static constexpr uint32_t REGS_ELEM = 168, REGS_DRAIN = 88, REGS_CTRL = 88;
 };
 static_assert(BwdPipe128Layout::SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+// Work item number w -> (key block, batch*head).  Items come in groups of
+// head_group heads (the last group may be smaller); inside a group, key block
+// 0 of every head first (the longest items when causal), then key block 1,
+// and so on.  A group's fp32 dQ rows are what the reduce-adds of its items
+// touch, so with the group small enough the accumulator rows being added
+// into stay in L2.
+__device__ __forceinline__ void bwd_item_decode(const BwdParams& p, int w, int& kblk, int& bh) {
+  const int per_group = p.head_group * p.n_blk;
+  const int gi = w / per_group, lw = w - gi * per_group;
+  const int first = gi * p.head_group;
+  const int hg = (p.BH - first) < p.head_group ? (p.BH - first) : p.head_group;
+  kblk = lw / hg;
+  bh = first + (lw - kblk * hg);
+}
+
+// Items of one CTA, taken from a list shared by all CTAs: the producer thread
+// claims the next item number with an atomic add on a counter in the
+// workspace (so CTAs that finish early take more items) and publishes it, one
+// item ahead of its own loads, in a ring of shared-memory slots; every other
+// role reads its items from the ring.  Same interface as BwdCursor.
+struct RingCursor {
+  BoundedWait wt;
+  uint32_t ring, full, empty;  // shared addresses: slot array, ITEM_FULL[0], ITEM_EMPTY[0]
+  bool uniform;                // called by whole warps (warp-uniform waits)
+  BwdParams p;
+  int r, kblk, bh, n, i0, i;
+  bool valid;
+  __device__ __forceinline__ void load() {
+    const int slot = r & 3;
+    const bool got = uniform ? wt.warp(full + 8u * slot, (r >> 2) & 1, 40) : wt(full + 8u * slot, (r >> 2) & 1, 40);
+    valid = false;
+    if (!got) return;  // the CTA is giving up: this role leaves its loop
+    int w;
+    asm volatile("ld.shared.s32 %0, [%1];" : "=r"(w) : "r"(ring + 4u * slot) : "memory");
+    mbar_arrive(empty + 8u * slot);
+    if (w < 0) return;
+    bwd_item_decode(p, w, kblk, bh);
+    n = p.causal ? (p.n_blk - kblk) : p.n_blk;
+    i0 = p.causal ? kblk : 0;
+    i = 0;
+    valid = true;
+  }
+  __device__ __forceinline__ void start() {
+    r = 0;
+    load();
+  }
+  __device__ __forceinline__ void next_block() {
+    if (++i >= n) {
+      ++r;
+      load();
+    }
+  }
+  __device__ __forceinline__ void next_item() {
+    ++r;
+    load();
+  }
+  __device__ __forceinline__ int qblk() const { return i0 + i; }
+};
 
 __global__ void __launch_bounds__(512, 1)
 fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -120,6 +187,10 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
     mbar_init(bar(L::ACC_FREE), 256);
     mbar_init(bar(L::DSTILE_FREE), 1);
     mbar_init(bar(L::TEARDOWN), 1);
+    for (int i = 0; i < L::RING; ++i) {
+      mbar_init(bar(L::ITEM_FULL + i), 1);
+      mbar_init(bar(L::ITEM_EMPTY + i), L::RING_READERS);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -156,8 +227,30 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      BwdCursor cur;
-      cur.start(p);
+      // the producer's own view of its items: it claims them and publishes
+      // them in the ring, one item ahead of its loads
+      struct PItem {
+        int r, kblk, bh, n, i0;
+        bool valid;
+      };
+      const int W = p.n_blk * p.BH;
+      auto publish = [&](int r, PItem& it) -> bool {
+        const int slot = r & 3;
+        if (r >= L::RING && !wait(bar(L::ITEM_EMPTY + slot), ((r - L::RING) >> 2) & 1, 41)) return false;
+        const int w = static_cast<int>(atomicAdd(p.item_ctr, 1u));
+        const int v = w < W ? w : -1;
+        asm volatile("st.shared.s32 [%0], %1;" ::"r"(base + L::RING_OFF + 4u * slot), "r"(v) : "memory");
+        mbar_arrive(bar(L::ITEM_FULL + slot));
+        it.r = r;
+        it.valid = v >= 0;
+        if (it.valid) {
+          bwd_item_decode(p, v, it.kblk, it.bh);
+          it.n = p.causal ? (p.n_blk - it.kblk) : p.n_blk;
+          it.i0 = p.causal ? it.kblk : 0;
+        }
+        return true;
+      };
+      PItem cur{}, nxt{};
       int g = 0, last_r = -1;
       int issued[NST];
       for (int s = 0; s < NST; ++s) issued[s] = -1;
@@ -174,8 +267,12 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
         issued[s] = gq;
         return true;
       };
-      bool ok = true;
-      for (; ok && cur.valid; cur.next_item()) {
+      bool ok = publish(0, cur);
+      for (; ok && cur.valid; cur = nxt) {
+        // the next item goes into the ring before this one's loads, so that
+        // the other roles never wait for it
+        ok = publish(cur.r + 1, nxt);
+        if (!ok) break;
         // the item's first query block goes ahead of its K/V, which must wait
         // for the previous item's products to release the K/V tiles; at the
         // cold start the rest of the ring waits until the first products'
@@ -224,8 +321,8 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
         }
         tc_commit(bar(L::DP_FULL));
       };
-      BwdCursor cur;
-      cur.start(p);
+      RingCursor cur{wait, base + L::RING_OFF, bar(L::ITEM_FULL), bar(L::ITEM_EMPTY), false, p};
+      cur.start();
       int g = 0;
       bool ok = true;
       for (; ok && cur.valid; cur.next_item()) {
@@ -296,8 +393,8 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float scale = p.scale;
     if (t == 0) tma_prefetch_desc(&tm_dq);
-    BwdCursor cur;
-    cur.start(p);
+    RingCursor cur{wait, base + L::RING_OFF, bar(L::ITEM_FULL), bar(L::ITEM_EMPTY), true, p};
+    cur.start();
     // A bounded wait that gives up only clears `ok`; the warpgroup leaves the
     // loop together at the AND vote on named barrier 2.
     bool ok = true;
@@ -374,8 +471,8 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
     // threads t < 64 the exponent offset and 1/l, threads t >= 64 delta.  The
     // raw values are loaded one block ahead (cursor pf).
     const int vq = t & 63, vrole = t >> 6;
-    BwdCursor pf;
-    pf.start(p);
+    RingCursor pf{wait, base + L::RING_OFF, bar(L::ITEM_FULL), bar(L::ITEM_EMPTY), true, p};
+    pf.start();
     auto fetch = [&](float& x, float& y) {
       x = 0.f;
       y = 0.f;
@@ -397,8 +494,8 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
     };
     float nx, ny;
     fetch(nx, ny);
-    BwdCursor cur;
-    cur.start(p);
+    RingCursor cur{wait, base + L::RING_OFF, bar(L::ITEM_FULL), bar(L::ITEM_EMPTY), true, p};
+    cur.start();
     int g = 0;
     // Error discipline as in the d = 64 kernel: the two warpgroups meet on
     // named barrier 1 once per block (an AND vote); a bounded wait that gives

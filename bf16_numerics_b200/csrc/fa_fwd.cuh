@@ -85,8 +85,8 @@ struct FwdLayout {
   static constexpr int Q_OFF = 0;                          // [QBUF][NT] tiles (also the O staging tiles)
   static constexpr int K_OFF = Q_OFF + QBUF * NT * TILE;   // [KVS] tiles
   static constexpr int V_OFF = K_OFF + KVS * TILE;         // [KVS] tiles
-  static constexpr int ALPHA_OFF = V_OFF + KVS * TILE;     // [NT][128] fp32 rescale factors
-  static constexpr int FIN_OFF = ALPHA_OFF + NT * 128 * 4; // [2 item slots][NT][4][128]: l, m, rm, rs
+  static constexpr int ALPHA_OFF = V_OFF + KVS * TILE;     // [2 slots][NT][128] fp32 rescale factors
+  static constexpr int FIN_OFF = ALPHA_OFF + 2 * NT * 128 * 4; // [2 item slots][NT][4][128]: l, m, rm, rs
   static constexpr int BAR_OFF = FIN_OFF + 2 * NT * 4 * 128 * 4;
   enum {
     Q_FULL = 0,                  // [2] by Q buffer
@@ -97,13 +97,15 @@ struct FwdLayout {
     V_EMPTY = V_FULL + 3,        // [3]
     S_FULL = V_EMPTY + 3,        // [2] by tile slot
     P_FULL = S_FULL + 2,         // [2]
-    ALPHA_READY = P_FULL + 2,    // [2]
-    CORR_DONE = ALPHA_READY + 2, // [2]
+    ALPHA_READY = P_FULL + 2,    // [2 factor slots][2 tile slots]
+    CORR_DONE = ALPHA_READY + 4, // [2]
     FIN_READY = CORR_DONE + 2,   // [2 item slots][2 tile slots]: one barrier per FIN slot, so
                                  // that a tile's softmax warps two items ahead stay one phase ahead
     O_DONE = FIN_READY + 4,      // [2]
     O_FREE = O_DONE + 2,         // [2]
-    TEARDOWN = O_FREE + 2,
+    S_FREE = O_FREE + 2,         // [2] separate-P mode: the softmax warps hold S in registers
+    PV_DONE = S_FREE + 2,        // [2] separate-P mode: a P_bar V product has completed
+    TEARDOWN = PV_DONE + 2,
     NBAR
   };
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base (4B), abort flag (4B)
@@ -111,14 +113,20 @@ struct FwdLayout {
   __host__ __device__ static constexpr uint32_t s_col(int t) { return 128u * t; }
   __host__ __device__ static constexpr uint32_t o_col(int t) { return 128u * NT + D * t; }
   __host__ __device__ static constexpr uint32_t olo_col(int t) { return 128u * NT + D * NT + D * t; }
+  // Separate-P mode (d = 64 without O_lo, where TMEM has room): P_bar gets its
+  // own 64 columns per tile after the O columns, so S of the next key tile can
+  // be computed while the softmax warps still work on this one.  Otherwise
+  // P_bar is written over the S columns it came from.
+  static constexpr bool SEPP = (D == 64 && !HP);
+  __host__ __device__ static constexpr uint32_t p_col(int t) { return SEPP ? 384u + 64u * t : 128u * t; }
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 512;
   // register budgets after setmaxnreg (launched with 128 per thread; the
-  // four warpgroups' shares add up to 4 x 128: 2 x 176 + 96 + 64 at d = 64,
+  // four warpgroups' shares add up to 4 x 128: 2 x 184 + 64 + 80 at d = 64,
   // 2 x 176 + 72 + 88 at d = 128, the splits at which no role spills)
-  static constexpr uint32_t REGS_SOFT = 176;
-  static constexpr uint32_t REGS_CORR = D == 64 ? 96 : 72;
-  static constexpr uint32_t REGS_CTRL = D == 64 ? 64 : 88;
+  static constexpr uint32_t REGS_SOFT = D == 64 ? 184 : 176;
+  static constexpr uint32_t REGS_CORR = D == 64 ? 64 : 72;
+  static constexpr uint32_t REGS_CTRL = D == 64 ? 80 : 88;
   static_assert(2 * REGS_SOFT + REGS_CORR + REGS_CTRL == 4 * 128, "register split");
 };
 static_assert(FwdLayout<64, false>::SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -191,7 +199,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_init(bar(L::S_FULL + t), 1);
       mbar_init(bar(L::P_FULL + t), 128);
       mbar_init(bar(L::ALPHA_READY + t), 128);
+      mbar_init(bar(L::ALPHA_READY + 2 + t), 128);
       mbar_init(bar(L::CORR_DONE + t), 128);
+      mbar_init(bar(L::S_FREE + t), 128);
+      mbar_init(bar(L::PV_DONE + t), 1);
       mbar_init(bar(L::FIN_READY + t), 128);
       mbar_init(bar(L::FIN_READY + 2 + t), 128);
       mbar_init(bar(L::O_DONE + t), 1);
@@ -318,8 +329,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // -------------------------------------------------------------- MMA issuer
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
-      // S_t = Q(buffer b, slot t) K(stage s)^T into slot t's S columns
-      auto issue_s = [&](int b, int t, int s) {
+      int ns[2] = {0, 0};  // S products issued per slot
+      // S_t = Q(buffer b, slot t) K(stage s)^T into slot t's S columns; in
+      // the separate-P mode once the softmax warps hold the previous S_t
+      auto issue_s = [&](int b, int t, int s) -> bool {
+        if constexpr (L::SEPP) {
+          if (ns[t] > 0 && !wait(bar(L::S_FREE + t), (ns[t] - 1) & 1, 12)) return false;
+          tc_fence_after();
+        }
+        ++ns[t];
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t koff = (ks >> 2) * L::HALF + (ks & 3) * 32;
@@ -327,6 +345,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                  sdesc_sw128(base + L::K_OFF + s * L::TILE + koff, 16, 1024), IDESC_S, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(L::S_FULL + t));
+        return true;
       };
       // O_t (+)= P_bar_t V(stage s)  (and O_lo_t (+)= P_lo_t V)
       auto issue_pv = [&](int t, int s, bool acc) {
@@ -334,7 +353,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
         for (int ks = 0; ks < L::BN / 16; ++ks) {
           const uint64_t bdesc = sdesc_sw128(vbase + ks * 2048, L::HALF, 1024);
-          mma_ts(tmem + L::o_col(t), tmem + L::s_col(t) + 8u * ks, bdesc, IDESC_O, (acc || ks > 0) ? 1u : 0u);
+          mma_ts(tmem + L::o_col(t), tmem + L::p_col(t) + 8u * ks, bdesc, IDESC_O, (acc || ks > 0) ? 1u : 0u);
         }
         if constexpr (HP) {
 #pragma unroll
@@ -358,7 +377,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           if (!wait(bar(L::K_FULL + s0), (gk / KVS) & 1, 5)) break;
           tc_fence_after();
           for (int t = 0; t < NT; ++t)
-            if (it.has(t)) issue_s(b, t, s0);
+            if (it.has(t) && !issue_s(b, t, s0)) ok = false;
+          if (!ok) break;
           tc_commit(bar(L::K_EMPTY + s0));
           FA_TRACE_POINT(10);
         }
@@ -366,6 +386,37 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           const int g = gk + j, sv = g % KVS;
           const bool next = j + 1 < nkv;
           const int sk = (g + 1) % KVS;
+          if constexpr (L::SEPP) {
+            // S of the next key tile first: it only needs the softmax warps to
+            // hold this step's S, and runs while they compute P_bar
+            if (next) {
+              if (!wait(bar(L::K_FULL + sk), ((g + 1) / KVS) & 1, 5)) { ok = false; break; }
+              for (int t = 0; t < NT; ++t)
+                if (it.has(t) && j + 1 < it.nkv[t] && !issue_s(b, t, sk)) ok = false;
+              if (!ok) break;
+              tc_commit(bar(L::K_EMPTY + sk));
+            }
+            if (!wait(bar(L::V_FULL + sv), (g / KVS) & 1, 8)) { ok = false; break; }
+            for (int t = 0; t < NT; ++t) {
+              if (!it.has(t) || j >= it.nkv[t]) continue;
+              if (!wait(bar(L::P_FULL + t), gs[t] & 1, 7)) { ok = false; break; }
+              if (j == 0) {
+                if (gi[t] > 0 && !wait(bar(L::O_FREE + t), (gi[t] - 1) & 1, 6)) { ok = false; break; }
+              } else {
+                if (!wait(bar(L::CORR_DONE + t), ga[t] & 1, 9)) { ok = false; break; }
+                ++ga[t];
+              }
+              tc_fence_after();
+              issue_pv(t, sv, j > 0);
+              tc_commit(bar(L::PV_DONE + t));
+              ++gs[t];
+              if (j + 1 == it.nkv[t]) ++gi[t];
+              FA_TRACE_POINT(11 + t);
+            }
+            if (!ok) break;
+            tc_commit(bar(L::V_EMPTY + sv));
+            continue;
+          }
           if (!wait(bar(L::V_FULL + sv), (g / KVS) & 1, 8)) { ok = false; break; }
           if (next && !wait(bar(L::K_FULL + sk), ((g + 1) / KVS) & 1, 5)) { ok = false; break; }
           for (int t = 0; t < NT; ++t) {
@@ -411,6 +462,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     FwdItem<NT> it;
     int n = 0;
     int ga[2] = {0, 0}, gi[2] = {0, 0};
+    int npv[2] = {0, 0};  // separate-P mode: P_bar V products of the slot before this item
     bool ok = true;
     for (; ok && it.load(p, n); ++n) {
       const int b = n % QBUF;
@@ -419,10 +471,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       for (int j = 1; ok && j < it.nkv_max(); ++j) {
         for (int t = 0; t < NT; ++t) {
           if (!it.has(t) || j >= it.nkv[t]) continue;
-          ok = wait.warp(bar(L::ALPHA_READY + t), ga[t] & 1, 15);
+          const int slot = ga[t] & 1;
+          ok = wait.warp(bar(L::ALPHA_READY + 2 * slot + t), (ga[t] >> 1) & 1, 15);
+          // separate-P mode: the previous step's product into O_t has completed
+          if constexpr (L::SEPP) ok = ok && wait.warp(bar(L::PV_DONE + t), (npv[t] + j - 1) & 1, 18);
           if (!ok) break;
           ++ga[t];
-          const float a = lds32(base + L::ALPHA_OFF + (t * 128 + r) * 4);
+          const float a = lds32(base + L::ALPHA_OFF + ((slot * NT + t) * 128 + r) * 4);
           if (__any_sync(0xffffffffu, a != 1.f)) {
             tc_fence_after();
 #pragma unroll 1
@@ -444,8 +499,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // epilogue of each tile of the item
       for (int t = 0; t < NT; ++t) {
         if (!it.has(t)) continue;
-        ok = wait.warp(bar(L::FIN_READY + 2 * (gi[t] & 1) + t), (gi[t] >> 1) & 1, 16) &&
-             wait.warp(bar(L::O_DONE + t), gi[t] & 1, 17);
+        ok = wait.warp(bar(L::FIN_READY + 2 * (gi[t] & 1) + t), (gi[t] >> 1) & 1, 16);
+        if constexpr (L::SEPP) {
+          ok = ok && wait.warp(bar(L::PV_DONE + t), (npv[t] + it.nkv[t] - 1) & 1, 17);
+          npv[t] += it.nkv[t];
+        } else {
+          ok = ok && wait.warp(bar(L::O_DONE + t), gi[t] & 1, 17);
+        }
         if (!ok) break;
         tc_fence_after();
         const uint32_t fin = base + L::FIN_OFF + ((((gi[t] & 1) * NT + t) * 4) * 128 + r) * 4;
@@ -523,7 +583,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const float beta = p.beta;
     const bool stall = t == 0 && inject_stall_here(1u);  // test hook (fa_debug_inject_stall)
     FwdItem<NT> it;
-    int n = 0, gs = 0, gi = 0;
+    int n = 0, gs = 0, gi = 0, na = 0;
     bool ok = true;
     for (; ok && (NT == 2 || t == 0) && it.load(p, n); ++n) {
       if (!it.has(t)) continue;
@@ -539,13 +599,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_after();
         float x[128];
         {
-          uint32_t r0[32], r1[32];
-          tmem_ld32x2(s_addr, s_addr + 32, r0, r1);
+          uint32_t raw[128];
+          tmem_ld32x4(s_addr, raw);  // four loads, one wait
 #pragma unroll
-          for (int c = 0; c < 32; ++c) { x[c] = __uint_as_float(r0[c]); x[32 + c] = __uint_as_float(r1[c]); }
-          tmem_ld32x2(s_addr + 64, s_addr + 96, r0, r1);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) { x[64 + c] = __uint_as_float(r0[c]); x[96 + c] = __uint_as_float(r1[c]); }
+          for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(raw[c]);
+        }
+        if constexpr (L::SEPP) {
+          // S is in registers: the next key tile's S may overwrite it
+          tc_fence_before();
+          mbar_arrive(bar(L::S_FREE + t));
         }
         // mask (diagonal tile / ragged tail); x[c] is key j*128 + c
         {
@@ -608,9 +670,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             alpha = ex2_approx((m_run - m_new) * kLog2e);
             l *= alpha;
           }
-          sts32(base + L::ALPHA_OFF + (t * 128 + r) * 4, alpha);
+          // two factor slots, used alternately: in the separate-P mode the
+          // softmax warps may run a step ahead of the correction warps
+          const int slot = na & 1;
+          sts32(base + L::ALPHA_OFF + ((slot * NT + t) * 128 + r) * 4, alpha);
           tc_fence_before();
-          mbar_arrive(bar(L::ALPHA_READY + t));
+          mbar_arrive(bar(L::ALPHA_READY + 2 * slot + t));
+          ++na;
         }
         m_run = m_new;
         if (r == 0) FA_TRACE_POINT(22 + t);
@@ -646,9 +712,19 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           f2_unpack(f2_add(sum2[0], sum2[1]), a, bsum);
           l += a + bsum;
         }
-        // P_bar over S columns [0,64) (and P_lo over [64,128)): S is in registers
-        tmem_st32(s_addr, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+        // P_bar over S columns [0,64) (and P_lo over [64,128)): S is in
+        // registers; in the separate-P mode into the slot's own P columns,
+        // once the previous P_bar V product has read them
+        const uint32_t p_addr = tmem + lane_base + L::p_col(t);
+        if constexpr (L::SEPP) {
+          if (gs > 0) {
+            ok = wait.warp(bar(L::PV_DONE + t), (gs - 1) & 1, 11);
+            if (!ok) break;
+            tc_fence_after();
+          }
+        }
+        tmem_st32(p_addr, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(p_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
         if constexpr (HP) {
           tmem_st32(s_addr + 64, *reinterpret_cast<const uint32_t(*)[32]>(&plo[0]));
           tmem_st32(s_addr + 96, *reinterpret_cast<const uint32_t(*)[32]>(&plo[32]));

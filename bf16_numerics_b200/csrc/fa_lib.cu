@@ -271,8 +271,16 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     if (!ensure_smem(fa::fa_bwd_main_pipe128_kernel, LP128::SMEM_BYTES, attr)) return FA_ERR_CUDA;
   }
   const long long rows = static_cast<long long>(BH) * N;
+  const int n_blk = (N + 127) / 128;
+  // workspace: delta | fp32 dQ accumulator | per-(bh, query block) counters
   float* delta = reinterpret_cast<float*>(ws);
-  float* dq_acc = reinterpret_cast<float*>(ws + round256(static_cast<size_t>(rows) * 4));
+  const size_t acc_off = round256(static_cast<size_t>(rows) * 4);
+  const size_t acc_bytes = static_cast<size_t>(rows) * D * 4;  // a multiple of 256
+  float* dq_acc = reinterpret_cast<float*>(ws + acc_off);
+  unsigned int* dq_cnt = reinterpret_cast<unsigned int*>(ws + acc_off + acc_bytes);
+  unsigned int* item_ctr = dq_cnt + static_cast<size_t>(BH) * n_blk;  // after the per-block counters
+  const long long clear_bytes =
+      static_cast<long long>(acc_bytes + round256((static_cast<size_t>(BH) * n_blk + 1) * 4));
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D) ||
       !make_map(&mdo, dO, BH, N, D))
@@ -283,10 +291,11 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     const dim3 grid(grid_for(rows, rows_per_block));
     cudaError_t e =
         o_is_hp ? launch_pdl(fa::fa_bwd_delta_kernel<D, float>, grid, dim3(256), 0, stream,
-                             static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows)
+                             static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows,
+                             clear_bytes)
                 : launch_pdl(fa::fa_bwd_delta_kernel<D, __nv_bfloat16>, grid, dim3(256), 0, stream,
                              static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta,
-                             dq_acc, rows);
+                             dq_acc, rows, clear_bytes);
     tm.done();
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("fa_bwd_delta_kernel launch", e);
@@ -297,11 +306,24 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.row_m = row_m;
     p.delta = delta;
     p.dq_acc = dq_acc;
+    p.dq_cnt = dq_cnt;
+    p.item_ctr = item_ctr;
+    // d = 128 item order: heads in groups whose fp32 dQ rows (N * D * 4 bytes
+    // per head) fit in 32 MB, a quarter of L2, so the reduce-adds of the items
+    // in flight hit L2
+    {
+      const long long per_head = static_cast<long long>(N) * D * 4;
+      long long hg = (32ll << 20) / (per_head > 0 ? per_head : 1);
+      if (hg < 1) hg = 1;
+      if (hg > BH) hg = BH;
+      p.head_group = static_cast<int>(hg);
+    }
+    p.dq = static_cast<__nv_bfloat16*>(dq);
     p.dk = static_cast<__nv_bfloat16*>(dk);
     p.dv = static_cast<__nv_bfloat16*>(dv);
     p.BH = BH;
     p.N = N;
-    p.n_blk = (N + 127) / 128;
+    p.n_blk = n_blk;
     p.causal = causal;
     p.mode = mode;
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
@@ -331,7 +353,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
     }
   }
-  {
+  if (D == 128) {
+    // (at d = 64 the main kernel converts each dQ block once it is complete)
     const long long n8 = rows * D / 8;
     LaunchTimer tm(FA_KERNEL_BWD_DQ, stream);
     cudaError_t e = launch_pdl(fa::fa_bwd_dq_convert_kernel, dim3(grid_for(n8, 256 * 4)), dim3(256), 0, stream,
@@ -372,7 +395,8 @@ size_t fa_bwd_workspace_dq_offset(int B, int H, int N, int d) {
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (!shape_ok(B, H, N, d) || (d != 64 && d != 128)) return 0;
   const size_t rows = static_cast<size_t>(B) * H * N;
-  return round256(rows * 4) + round256(rows * static_cast<size_t>(d) * 4);
+  const size_t blocks = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128);
+  return round256(rows * 4) + round256(rows * static_cast<size_t>(d) * 4) + round256((blocks + 1) * 4);
 }
 
 }  // extern "C"

@@ -215,6 +215,28 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t taddr0, uint32_t taddr1, ui
       : "r"(taddr0), "r"(taddr1));
 #undef FA_S8
 }
+// 32 lanes x 128 columns: four 32-column loads and one wait.  The loads
+// leave their registers undefined until the wait; the wait names all 128 as
+// in/out operands, so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : FA_R8(0), FA_R8(8), FA_R8(16), FA_R8(24)
+      : "r"(taddr));
+}
+#define FA_U8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
+__device__ __forceinline__ void tmem_ld32x4(uint32_t taddr, uint32_t (&r)[128]) {
+  tmem_ld32_nowait(taddr, &r[0]);
+  tmem_ld32_nowait(taddr + 32, &r[32]);
+  tmem_ld32_nowait(taddr + 64, &r[64]);
+  tmem_ld32_nowait(taddr + 96, &r[96]);
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : FA_U8(0), FA_U8(8), FA_U8(16), FA_U8(24), FA_U8(32), FA_U8(40), FA_U8(48), FA_U8(56), FA_U8(64),
+                 FA_U8(72), FA_U8(80), FA_U8(88), FA_U8(96), FA_U8(104), FA_U8(112), FA_U8(120));
+}
+#undef FA_U8
 #undef FA_R8
 
 #define FA_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
@@ -309,6 +331,13 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // wait until every committed bulk group has completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// wait until at most N committed bulk groups are still in flight (complete,
+// not only read)
+template <int N>
+__device__ __forceinline__ void bulk_wait_allow() { asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory"); }
+// async-proxy writes to global memory (completed bulk operations) -> ordered
+// before this thread's later generic-proxy accesses and fences
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 // wait until at most one committed bulk group is still in flight
 __device__ __forceinline__ void bulk_wait_all_but_one() { asm volatile("cp.async.bulk.wait_group 1;" ::: "memory"); }
 }  // namespace fa
