@@ -34,8 +34,8 @@ namespace fa {
 
 // ------------------------------------------------------------------ delta
 // delta[r] = sum_c dO[r,c] * O[r,c] in fp32; also clears the dQ accumulator
-// and the per-block completion counters behind it (with TMA bulk stores of a
-// zeroed shared-memory buffer).  O is the bf16 output of the forward, or (OT = float) its fp32 value
+// and the work-item counter behind it (with TMA bulk stores of a zeroed
+// shared-memory buffer).  O is the bf16 output of the forward, or (OT = float) its fp32 value
 // before rounding (the high-precision O_hp of the pages).
 // Memory bound: each row of O and dO is read once with 16-byte loads, LPR
 // lanes per row (8 elements of dO per lane); every warp takes U row groups at
@@ -111,7 +111,7 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
   grid_dependency_wait();  // O comes from the forward grid; the workspace may be the previous grid's
   if (threadIdx.x == 0) {
     // this block's share of the region to clear (the fp32 dQ accumulator and
-    // the completion counters that follow it; a multiple of 256 bytes):
+    // the work-item counter that follows it; a multiple of 256 bytes):
     // 16 KB chunks dealt round-robin over the blocks
     const long long bytes = clear_bytes;
     const long long nchunk = (bytes + ZCHUNK - 1) / ZCHUNK;
@@ -190,10 +190,8 @@ struct BwdParams {
   const float* row_m;  // [BH, N], stabilised mode only
   const float* delta;  // [BH, N]
   float* dq_acc;       // [BH, N, D] fp32, zeroed by the delta kernel
-  unsigned int* dq_cnt;  // [BH, n_blk] contributions added so far, zeroed by the delta kernel
   unsigned int* item_ctr;  // d = 128: next unclaimed work item (zeroed by the delta kernel)
   int head_group;          // d = 128: heads per group of the item order
-  __nv_bfloat16* dq;   // [BH, N, D] (written by the main kernel at d = 64)
   __nv_bfloat16* dk;   // [BH, N, D]
   __nv_bfloat16* dv;   // [BH, N, D]
   int BH, N, n_blk;

@@ -16,23 +16,17 @@
 //     a key row: warpgroup h takes columns [64h, 64h+64).  Both copy their S^T
 //     columns to registers and meet at a named barrier; then warpgroup h
 //     writes its bf16 P^T into S^T cols [32h, 32h+32), so P^T occupies
-//     [0,64) and [64,128) is free for dQ.  Once they hold dP^T in registers
-//     they release its columns, so dP^T of the next block is computed while
-//     they form dS.
-//   * dS goes to shared memory only: a double-buffered [keys][queries] bf16
-//     tile (128B-swizzled, two 64-query halves) that is the A operand of both
-//     dK += dS^T Q (read K-major) and dQ_g = dS K (read MN-major).  dQ_g is
-//     one N = 64 product into S^T cols [64,128) of the block's S^T buffer,
-//     which no later product of the block touches.
+//     [0,64) and [64,128) is free for dQ.  dS^T goes into the first half of
+//     the dP^T columns each warpgroup has just read (64h + [0,32)), which
+//     needs no barrier.
+//   * dQ_g = dS K is one N = 64 product into S^T cols [64,128) of the same
+//     buffer, which no later product of the block touches.
 //   * Four drain warps move the dQ partial from TMEM into a 128B-swizzled
 //     fp32 staging box in shared memory and add it to the fp32 accumulator in
 //     global memory with one TMA tensor reduce-add per 32-column half, one
 //     half after the other through the same box (rows past N are clipped by
-//     the tensor map).  Two blocks later, once those reduce-adds are
-//     complete, they count the contribution on the query block's counter;
-//     the CTA that completes a query block converts it to bf16 dQ.  They
-//     also prepare the per-query vectors (lse or m, 1/l, delta) two blocks
-//     ahead.
+//     the tensor map).  They also prepare the per-query
+//     vectors (lse or m, 1/l, delta) two blocks ahead.
 //
 // Barrier phases count a global query-block index g that runs across the
 // CTA's items; every phase of every barrier is waited for in order and no
@@ -56,8 +50,8 @@ struct BwdPipeLayout {
   static constexpr int D = 64, B = 128, TILE = 128 * 64 * 2, NST = 3;
   static constexpr int K_OFF = 0, V_OFF = TILE, Q_OFF = 2 * TILE;
   static constexpr int DO_OFF = Q_OFF + NST * TILE;
-  static constexpr int DS_OFF = DO_OFF + NST * TILE;  // [2 buffers] dS^T [keys][queries], two 64-query halves
-  static constexpr int DQS_OFF = DS_OFF + 4 * TILE;   // dQ staging: one [128 rows][32 fp32] swizzled box
+  static constexpr int DS_OFF = DO_OFF + NST * TILE;  // dS^T [keys][queries], two 64-query halves
+  static constexpr int DQS_OFF = DS_OFF + 2 * TILE;   // dQ staging: one [128 rows][32 fp32] swizzled box
   static constexpr int VEC_OFF = DQS_OFF + TILE;      // [2 stages][3][128] fp32
   static constexpr int BAR_OFF = VEC_OFF + 2 * 3 * 128 * 4;
   enum {
@@ -68,7 +62,6 @@ struct BwdPipeLayout {
     S_FULL = Q_EMPTY + NST,    // [2]
     P_FULL = S_FULL + 2,       // [2]
     DP_FULL = P_FULL + 2,
-    DP_FREE,                   // the elementwise warps hold dP^T of the block in registers
     DS_FULL,
     DQ_FULL,                   // [2]
     DQ_FREE = DQ_FULL + 2,
@@ -85,7 +78,6 @@ struct BwdPipeLayout {
   static constexpr int THREADS = 512;
   static constexpr uint32_t REGS_ELEM = 168, REGS_DRAIN = 88, REGS_CTRL = 88;
 };
-static_assert(BwdPipeLayout::SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int x, int y, int z) {
   asm volatile(
@@ -172,7 +164,6 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       mbar_init(bar(L::VEC_EMPTY + b), 256);
     }
     mbar_init(bar(L::DP_FULL), 1);
-    mbar_init(bar(L::DP_FREE), 256);
     mbar_init(bar(L::DS_FULL), 256);
     mbar_init(bar(L::DQ_FREE), 128);
     mbar_init(bar(L::ACC_DONE), 1);
@@ -289,9 +280,6 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (!wait(bar(L::Q_FULL + (g0 % NST)), (g0 / NST) & 1, 3)) break;
         tc_fence_after();
         issue_s(g0);
-        // dP^T of the previous block has been copied to registers
-        if (g0 > 0 && !wait(bar(L::DP_FREE), (g0 - 1) & 1, 10)) break;
-        tc_fence_after();
         issue_dp(g0);
         if (n > 1) {
           if (!wait(bar(L::Q_FULL + ((g0 + 1) % NST)), ((g0 + 1) / NST) & 1, 3)) break;
@@ -311,30 +299,26 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           for (int ks = 0; ks < 8; ++ks)
             mma_ts(tmem + L::DV_COL, tmem + 128u * b + 8u * ks, sdesc_sw128(do_tile(g) + ks * 2048, 16384, 1024),
                    IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
-          // dP^T of the next block as soon as this block's dP^T is in registers
-          // (its Q/dO stage was waited for when S^T of that block was issued)
-          if (i + 1 < n) {
-            if (!wait(bar(L::DP_FREE), g & 1, 10)) { ok = false; break; }
-            tc_fence_after();
-            issue_dp(g + 1);
-          }
           if (!wait(bar(L::DS_FULL), g & 1, 5)) { ok = false; break; }
           FA_TRACE_POINT(11);
           tc_fence_after();
-          const uint32_t ds_tile = base + L::DS_OFF + 2 * b * TILE;
-          // dK += dS^T Q_g   (A: dS^T [keys][queries] in shared memory, K-major)
+          // dK += dS^T Q_g
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t a = tmem + L::DPT_COL + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4));
+            mma_ts(tmem + L::DK_COL, a, sdesc_sw128(q_tile(g) + ks * 2048, 16384, 1024), IDESC_KV,
+                   (i > 0 || ks > 0) ? 1u : 0u);
+          }
+          // dQ_g = dS K into S^T cols [64,128) of the same buffer
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + L::DK_COL, sdesc_sw128(ds_tile + (ks >> 2) * TILE + (ks & 3) * 32, 16, 1024),
-                   sdesc_sw128(q_tile(g) + ks * 2048, 16384, 1024), IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
-          // dQ_g = dS K into S^T cols [64,128) of the same buffer (A: the same tile, MN-major)
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + 128u * b + 64u, sdesc_sw128(ds_tile + ks * 2048, TILE, 1024),
+            mma_ss(tmem + 128u * b + 64u, sdesc_sw128(base + L::DS_OFF + ks * 2048, 16384, 1024),
                    sdesc_sw128(base + L::K_OFF + ks * 2048, 16384, 1024), IDESC_DQ, ks > 0 ? 1u : 0u);
           tc_commit(bar(L::DQ_FULL + b));
           tc_commit(bar(L::Q_EMPTY + (g % NST)));
-          if (i + 1 == n) {
+          if (i + 1 < n) {
+            issue_dp(g + 1);
+          } else {
             tc_commit(bar(L::ACC_DONE));  // dV, dK of this item complete
             tc_commit(bar(L::KV_EMPTY));  // K, V of this item no longer read
           }
@@ -405,50 +389,11 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     for (int k = 0; k < 2 && pub.valid; ++k, ++g_pub, pub.next_block()) publish_vec(g_pub, pub, load_vec(pub));
     Vec3 nxt = load_vec(pub);
     if (t == 0) tma_prefetch_desc(&tm_dq);
-    // dQ conversion in this kernel: after a block's reduce-adds are complete
-    // (checked two blocks later, so the drain does not stall on them), thread
-    // 0 counts that contribution on the query block's counter; the CTA whose
-    // count completes the block (query block qb has qb+1 contributions when
-    // causal, n_blk otherwise) converts its 128 rows to bf16.  The decision
-    // is broadcast through two flag slots used alternately, so one barrier
-    // per block suffices.
-    volatile int* conv_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
-    int n_counted = 0;
-    auto count_and_convert = [&](int bh, int qb) {
-      if (t == 0) {
-        fence_proxy_async_global();  // the completed reduce-adds, before the count
-        __threadfence();
-        const unsigned expected = static_cast<unsigned>(p.causal ? qb + 1 : p.n_blk);
-        const unsigned old = atomicAdd(p.dq_cnt + static_cast<size_t>(bh) * p.n_blk + qb, 1u);
-        __threadfence();
-        conv_flag[n_counted & 1] = (old + 1 == expected) ? 1 : 0;
-      }
-      named_barrier_sync(2, 128);
-      const bool last = conv_flag[n_counted & 1] != 0;
-      ++n_counted;
-      const int q = qb * L::B + t;
-      if (last && q < p.N) {
-        const size_t ri = static_cast<size_t>(bh) * p.N + q;
-        const float4* src = reinterpret_cast<const float4*>(p.dq_acc + ri * L::D);
-        uint4* dst = reinterpret_cast<uint4*>(p.dq + ri * L::D);
-        float4 a[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) a[c] = __ldcg(src + c);  // L2: written by other CTAs' reduce-adds
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          dst[c] = make_uint4(pack_bf16x2(a[2 * c].x, a[2 * c].y), pack_bf16x2(a[2 * c].z, a[2 * c].w),
-                              pack_bf16x2(a[2 * c + 1].x, a[2 * c + 1].y),
-                              pack_bf16x2(a[2 * c + 1].z, a[2 * c + 1].w));
-      }
-    };
-    // (batch*head, query block) of the last two blocks not yet counted
-    int pend_bh[2] = {0, 0}, pend_qb[2] = {0, 0};
     // A bounded wait that gives up only clears `ok`; the warpgroup leaves the
     // loop together at the AND vote on named barrier 2 (a stale TMEM read
     // before it is in bounds and harmless).
-    bool ok = true, aborted = false;
-    int g = 0;
-    for (; cur.valid; ++g, cur.next_block()) {
+    bool ok = true;
+    for (int g = 0; cur.valid; ++g, cur.next_block()) {
       const int b = g & 1;
       {
         // every lane calls the warp-uniform wait (ok may differ per lane here)
@@ -462,7 +407,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       tc_fence_before();
       mbar_arrive(bar(L::DQ_FREE));
       if (t == 0) bulk_wait_read_all();  // the previous reduce has finished reading the staging tile
-      if (!named_barrier_and(2, 128, ok)) { aborted = true; break; }
+      if (!named_barrier_and(2, 128, ok)) break;
       // row t of the 32-column box, 16-byte chunk c stored at chunk c ^ (t & 7);
       // the two halves of the row go through the box one after the other
       const uint32_t row = base + L::DQS_OFF + t * 128;
@@ -488,14 +433,6 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         }
       }
       if (t == 0) FA_TRACE_POINT(31);
-      // block g-2's two reduce-add groups are complete once at most four
-      // (blocks g-1 and g) are pending
-      if (g >= 2) {
-        if (t == 0) bulk_wait_allow<4>();
-        count_and_convert(pend_bh[b], pend_qb[b]);
-      }
-      pend_bh[b] = cur.bh;
-      pend_qb[b] = cur.qblk();
       if (pub.valid) {
         // block g+2 reuses the vector stage of block g
         // (a wait that gives up skips the publish; the next vote ends the loop)
@@ -509,11 +446,6 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       }
     }
     if (t == 0) bulk_wait_all();
-    if (!aborted) {
-      // the last two blocks
-      if (g >= 2) count_and_convert(pend_bh[g & 1], pend_qb[g & 1]);
-      if (g >= 1) count_and_convert(pend_bh[(g - 1) & 1], pend_qb[(g - 1) & 1]);
-    }
     teardown();
     return;
   }
@@ -529,7 +461,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     const uint64_t C2 = f2_pack(c_log2, c_log2);
     const bool mode1 = p.mode == 1;
     const int qoff = 64 * h;
-
+    const uint32_t ds_row = base + L::DS_OFF + h * TILE + t * 128;
     BwdCursor cur;
     cur.start(p);
     int g = 0;
@@ -605,6 +537,8 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (threadIdx.x == 0) FA_TRACE_POINT(21);
         ok = wait.warp(bar(L::DP_FULL), g & 1, 10);
         if (threadIdx.x == 0) FA_TRACE_POINT(22);
+        // the dQ product of the previous block has finished reading the dS tile
+        ok = ok && (g == 0 || wait.warp(bar(L::DQ_FULL + ((g - 1) & 1)), ((g - 1) >> 1) & 1, 11));
         if (!ok) continue;  // the next meeting takes everyone out
         tc_fence_after();
         uint32_t dpr[64];
@@ -614,9 +548,6 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           tmem_ld32x2(tmem + lane_base + L::DPT_COL + 64u * h, tmem + lane_base + L::DPT_COL + 64u * h + 32u, d0,
                       d1);
         }
-        // the dP^T columns may take the next block's product
-        tc_fence_before();
-        mbar_arrive(bar(L::DP_FREE));
         uint32_t dk_[32];
 #pragma unroll
         for (int pi = 0; pi < 32; pi += 2) {
@@ -633,19 +564,16 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           dk_[pi] = pack_bf16x2(d0, d1);
           dk_[pi + 1] = pack_bf16x2(d2, d3);
         }
-        // dS buffer b was last read by the dK and dQ products of block g-2
-        const bool buf_free = g < 2 || wait.warp(bar(L::DQ_FULL + b), ((g - 2) >> 1) & 1, 11);
-        ok = ok && buf_free;
+        // dS^T into the dP^T columns this warpgroup has read: 64h + [0,32)
+        tmem_st32(tmem + lane_base + L::DPT_COL + 64u * h, dk_);
         // dS^T row t, queries 64h + [0,64) = the eight 16-byte chunks of the half tile's row
-        // (after a wait that gave up, skip the write; the next vote takes everyone out)
-        if (buf_free) {
-          const uint32_t ds_row = base + L::DS_OFF + (2 * b + h) * TILE + t * 128;
 #pragma unroll
-          for (int chunk = 0; chunk < 8; ++chunk)
-            sts128(ds_row + ((chunk ^ (t & 7)) << 4), dk_[4 * chunk], dk_[4 * chunk + 1], dk_[4 * chunk + 2],
-                   dk_[4 * chunk + 3]);
-        }
+        for (int chunk = 0; chunk < 8; ++chunk)
+          sts128(ds_row + ((chunk ^ (t & 7)) << 4), dk_[4 * chunk], dk_[4 * chunk + 1], dk_[4 * chunk + 2],
+                 dk_[4 * chunk + 3]);
         fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
         mbar_arrive(bar(L::DS_FULL));
         mbar_arrive(bar(L::VEC_EMPTY + b));
         if (threadIdx.x == 0) FA_TRACE_POINT(24);

@@ -140,13 +140,17 @@ struct RingCursor {
     r = 0;
     load();
   }
+  // Past the end of the list the cursor stays where it is: the slot after the
+  // end marker is never published (the vector prefetch cursor, which runs two
+  // blocks ahead, keeps advancing after the end).
   __device__ __forceinline__ void next_block() {
-    if (++i >= n) {
+    if (valid && ++i >= n) {
       ++r;
       load();
     }
   }
   __device__ __forceinline__ void next_item() {
+    if (!valid) return;
     ++r;
     load();
   }

@@ -13,7 +13,14 @@
 // P_bar operand is computed against the shift in force for the rows seen so
 // far (the final shift once the last tile has been merged).
 //
-// Persistent kernel, one CTA per SM.  A work item is a pair of 128-row Q tiles
+// This file holds the method's formulas and parameters for every forward
+// kernel, and the pair kernel that runs head dimension 128 (head dimension 64
+// runs the column-split kernel of fa_fwd_split.cuh, which hides the latency
+// of the per-tile chain better at that size: 43 us against 47 us for this
+// kernel on g2s; at d = 128 this one is faster, 658 us against 823 us on the
+// long workload).
+//
+// Pair kernel: persistent, one CTA per SM.  A work item is a pair of 128-row Q tiles
 // of one (batch, head) -- tile slot 0 the longer one (causal: query blocks
 // n-1-2p and n-2-2p of n) -- which share every K and V tile they both see;
 // items are ordered longest first and dealt to the CTAs in snake order (round
@@ -103,9 +110,7 @@ struct FwdLayout {
                                  // that a tile's softmax warps two items ahead stay one phase ahead
     O_DONE = FIN_READY + 4,      // [2]
     O_FREE = O_DONE + 2,         // [2]
-    S_FREE = O_FREE + 2,         // [2] separate-P mode: the softmax warps hold S in registers
-    PV_DONE = S_FREE + 2,        // [2] separate-P mode: a P_bar V product has completed
-    TEARDOWN = PV_DONE + 2,
+    TEARDOWN = O_FREE + 2,
     NBAR
   };
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base (4B), abort flag (4B)
@@ -113,26 +118,17 @@ struct FwdLayout {
   __host__ __device__ static constexpr uint32_t s_col(int t) { return 128u * t; }
   __host__ __device__ static constexpr uint32_t o_col(int t) { return 128u * NT + D * t; }
   __host__ __device__ static constexpr uint32_t olo_col(int t) { return 128u * NT + D * NT + D * t; }
-  // Separate-P mode (d = 64 without O_lo, where TMEM has room): P_bar gets its
-  // own 64 columns per tile after the O columns, so S of the next key tile can
-  // be computed while the softmax warps still work on this one.  Otherwise
-  // P_bar is written over the S columns it came from.
-  static constexpr bool SEPP = (D == 64 && !HP);
-  __host__ __device__ static constexpr uint32_t p_col(int t) { return SEPP ? 384u + 64u * t : 128u * t; }
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 512;
   // register budgets after setmaxnreg (launched with 128 per thread; the
-  // four warpgroups' shares add up to 4 x 128: 2 x 184 + 64 + 80 at d = 64,
-  // 2 x 176 + 72 + 88 at d = 128, the splits at which no role spills)
-  static constexpr uint32_t REGS_SOFT = D == 64 ? 184 : 176;
-  static constexpr uint32_t REGS_CORR = D == 64 ? 64 : 72;
-  static constexpr uint32_t REGS_CTRL = D == 64 ? 80 : 88;
+  // four warpgroups' shares add up to 4 x 128: 2 x 176 + 72 + 88, the split
+  // at which no role spills at d = 128)
+  static constexpr uint32_t REGS_SOFT = 176, REGS_CORR = 72, REGS_CTRL = 88;
   static_assert(2 * REGS_SOFT + REGS_CORR + REGS_CTRL == 4 * 128, "register split");
 };
-static_assert(FwdLayout<64, false>::SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(FwdLayout<128, false>::SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(FwdLayout<128, true>::SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(FwdLayout<64, true>::olo_col(1) + 64 <= 512 && FwdLayout<128, true>::olo_col(0) + 128 <= 512,
+static_assert(FwdLayout<128, false>::o_col(1) + 128 <= 512 && FwdLayout<128, true>::olo_col(0) + 128 <= 512,
               "TMEM budget");
 
 // One work item: NT Q tiles of one (batch, head).  Slot 0 always holds a
@@ -201,8 +197,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_init(bar(L::ALPHA_READY + t), 128);
       mbar_init(bar(L::ALPHA_READY + 2 + t), 128);
       mbar_init(bar(L::CORR_DONE + t), 128);
-      mbar_init(bar(L::S_FREE + t), 128);
-      mbar_init(bar(L::PV_DONE + t), 1);
       mbar_init(bar(L::FIN_READY + t), 128);
       mbar_init(bar(L::FIN_READY + 2 + t), 128);
       mbar_init(bar(L::O_DONE + t), 1);
@@ -329,15 +323,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // -------------------------------------------------------------- MMA issuer
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
-      int ns[2] = {0, 0};  // S products issued per slot
-      // S_t = Q(buffer b, slot t) K(stage s)^T into slot t's S columns; in
-      // the separate-P mode once the softmax warps hold the previous S_t
-      auto issue_s = [&](int b, int t, int s) -> bool {
-        if constexpr (L::SEPP) {
-          if (ns[t] > 0 && !wait(bar(L::S_FREE + t), (ns[t] - 1) & 1, 12)) return false;
-          tc_fence_after();
-        }
-        ++ns[t];
+      // S_t = Q(buffer b, slot t) K(stage s)^T into slot t's S columns
+      auto issue_s = [&](int b, int t, int s) {
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t koff = (ks >> 2) * L::HALF + (ks & 3) * 32;
@@ -345,7 +332,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                  sdesc_sw128(base + L::K_OFF + s * L::TILE + koff, 16, 1024), IDESC_S, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(L::S_FULL + t));
-        return true;
       };
       // O_t (+)= P_bar_t V(stage s)  (and O_lo_t (+)= P_lo_t V)
       auto issue_pv = [&](int t, int s, bool acc) {
@@ -353,7 +339,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
         for (int ks = 0; ks < L::BN / 16; ++ks) {
           const uint64_t bdesc = sdesc_sw128(vbase + ks * 2048, L::HALF, 1024);
-          mma_ts(tmem + L::o_col(t), tmem + L::p_col(t) + 8u * ks, bdesc, IDESC_O, (acc || ks > 0) ? 1u : 0u);
+          mma_ts(tmem + L::o_col(t), tmem + L::s_col(t) + 8u * ks, bdesc, IDESC_O, (acc || ks > 0) ? 1u : 0u);
         }
         if constexpr (HP) {
 #pragma unroll
@@ -377,8 +363,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           if (!wait(bar(L::K_FULL + s0), (gk / KVS) & 1, 5)) break;
           tc_fence_after();
           for (int t = 0; t < NT; ++t)
-            if (it.has(t) && !issue_s(b, t, s0)) ok = false;
-          if (!ok) break;
+            if (it.has(t)) issue_s(b, t, s0);
           tc_commit(bar(L::K_EMPTY + s0));
           FA_TRACE_POINT(10);
         }
@@ -386,37 +371,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           const int g = gk + j, sv = g % KVS;
           const bool next = j + 1 < nkv;
           const int sk = (g + 1) % KVS;
-          if constexpr (L::SEPP) {
-            // S of the next key tile first: it only needs the softmax warps to
-            // hold this step's S, and runs while they compute P_bar
-            if (next) {
-              if (!wait(bar(L::K_FULL + sk), ((g + 1) / KVS) & 1, 5)) { ok = false; break; }
-              for (int t = 0; t < NT; ++t)
-                if (it.has(t) && j + 1 < it.nkv[t] && !issue_s(b, t, sk)) ok = false;
-              if (!ok) break;
-              tc_commit(bar(L::K_EMPTY + sk));
-            }
-            if (!wait(bar(L::V_FULL + sv), (g / KVS) & 1, 8)) { ok = false; break; }
-            for (int t = 0; t < NT; ++t) {
-              if (!it.has(t) || j >= it.nkv[t]) continue;
-              if (!wait(bar(L::P_FULL + t), gs[t] & 1, 7)) { ok = false; break; }
-              if (j == 0) {
-                if (gi[t] > 0 && !wait(bar(L::O_FREE + t), (gi[t] - 1) & 1, 6)) { ok = false; break; }
-              } else {
-                if (!wait(bar(L::CORR_DONE + t), ga[t] & 1, 9)) { ok = false; break; }
-                ++ga[t];
-              }
-              tc_fence_after();
-              issue_pv(t, sv, j > 0);
-              tc_commit(bar(L::PV_DONE + t));
-              ++gs[t];
-              if (j + 1 == it.nkv[t]) ++gi[t];
-              FA_TRACE_POINT(11 + t);
-            }
-            if (!ok) break;
-            tc_commit(bar(L::V_EMPTY + sv));
-            continue;
-          }
           if (!wait(bar(L::V_FULL + sv), (g / KVS) & 1, 8)) { ok = false; break; }
           if (next && !wait(bar(L::K_FULL + sk), ((g + 1) / KVS) & 1, 5)) { ok = false; break; }
           for (int t = 0; t < NT; ++t) {
@@ -462,7 +416,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     FwdItem<NT> it;
     int n = 0;
     int ga[2] = {0, 0}, gi[2] = {0, 0};
-    int npv[2] = {0, 0};  // separate-P mode: P_bar V products of the slot before this item
     bool ok = true;
     for (; ok && it.load(p, n); ++n) {
       const int b = n % QBUF;
@@ -473,8 +426,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           if (!it.has(t) || j >= it.nkv[t]) continue;
           const int slot = ga[t] & 1;
           ok = wait.warp(bar(L::ALPHA_READY + 2 * slot + t), (ga[t] >> 1) & 1, 15);
-          // separate-P mode: the previous step's product into O_t has completed
-          if constexpr (L::SEPP) ok = ok && wait.warp(bar(L::PV_DONE + t), (npv[t] + j - 1) & 1, 18);
           if (!ok) break;
           ++ga[t];
           const float a = lds32(base + L::ALPHA_OFF + ((slot * NT + t) * 128 + r) * 4);
@@ -499,13 +450,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // epilogue of each tile of the item
       for (int t = 0; t < NT; ++t) {
         if (!it.has(t)) continue;
-        ok = wait.warp(bar(L::FIN_READY + 2 * (gi[t] & 1) + t), (gi[t] >> 1) & 1, 16);
-        if constexpr (L::SEPP) {
-          ok = ok && wait.warp(bar(L::PV_DONE + t), (npv[t] + it.nkv[t] - 1) & 1, 17);
-          npv[t] += it.nkv[t];
-        } else {
-          ok = ok && wait.warp(bar(L::O_DONE + t), gi[t] & 1, 17);
-        }
+        ok = wait.warp(bar(L::FIN_READY + 2 * (gi[t] & 1) + t), (gi[t] >> 1) & 1, 16) &&
+             wait.warp(bar(L::O_DONE + t), gi[t] & 1, 17);
         if (!ok) break;
         tc_fence_after();
         const uint32_t fin = base + L::FIN_OFF + ((((gi[t] & 1) * NT + t) * 4) * 128 + r) * 4;
@@ -604,11 +550,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
           for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(raw[c]);
         }
-        if constexpr (L::SEPP) {
-          // S is in registers: the next key tile's S may overwrite it
-          tc_fence_before();
-          mbar_arrive(bar(L::S_FREE + t));
-        }
         // mask (diagonal tile / ragged tail); x[c] is key j*128 + c
         {
           const int kv0 = j * L::BN;
@@ -670,8 +611,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             alpha = ex2_approx((m_run - m_new) * kLog2e);
             l *= alpha;
           }
-          // two factor slots, used alternately: in the separate-P mode the
-          // softmax warps may run a step ahead of the correction warps
+          // two factor slots, used alternately (one slot would also do here:
+          // the next factor is written after S of the next step, which needs
+          // this step's P_bar V, which needs the correction warps' hand-back)
           const int slot = na & 1;
           sts32(base + L::ALPHA_OFF + ((slot * NT + t) * 128 + r) * 4, alpha);
           tc_fence_before();
@@ -712,19 +654,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           f2_unpack(f2_add(sum2[0], sum2[1]), a, bsum);
           l += a + bsum;
         }
-        // P_bar over S columns [0,64) (and P_lo over [64,128)): S is in
-        // registers; in the separate-P mode into the slot's own P columns,
-        // once the previous P_bar V product has read them
-        const uint32_t p_addr = tmem + lane_base + L::p_col(t);
-        if constexpr (L::SEPP) {
-          if (gs > 0) {
-            ok = wait.warp(bar(L::PV_DONE + t), (gs - 1) & 1, 11);
-            if (!ok) break;
-            tc_fence_after();
-          }
-        }
-        tmem_st32(p_addr, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(p_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+        // P_bar over S columns [0,64) (and P_lo over [64,128)): S is in registers
+        tmem_st32(s_addr, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
         if constexpr (HP) {
           tmem_st32(s_addr + 64, *reinterpret_cast<const uint32_t(*)[32]>(&plo[0]));
           tmem_st32(s_addr + 96, *reinterpret_cast<const uint32_t(*)[32]>(&plo[32]));

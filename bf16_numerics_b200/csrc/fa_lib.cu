@@ -16,6 +16,7 @@
 #include "fa_b200.h"
 #include "fa_bwd_pipe.cuh"
 #include "fa_bwd_pipe128.cuh"
+#include "fa_fwd_split.cuh"
 
 namespace {
 
@@ -220,29 +221,46 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   p.mode = mode;
   p.beta = beta;
   p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
-  // persistent: one CTA per SM (at most one per work item; an item is
-  // FwdLayout::NT Q tiles of one (batch, head))
+  // persistent grids: at most one CTA per work item
   const int n_sm = sm_count();
   if (n_sm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)");
-  auto launch = [&](auto kernel, int smem, int nt) {
+  // items of nt Q tiles, ctas_per_sm CTAs of `threads` threads per SM
+  auto launch = [&](auto kernel, int smem, int nt, int ctas_per_sm, int threads) {
     const long long items = static_cast<long long>((p.n_qblk + nt - 1) / nt) * BH;
-    const unsigned grid = static_cast<unsigned>(items < n_sm ? items : n_sm);
+    const long long slots = static_cast<long long>(n_sm) * ctas_per_sm;
+    const unsigned grid = static_cast<unsigned>(items < slots ? items : slots);
     LaunchTimer tm(FA_KERNEL_FWD, stream);
-    const cudaError_t err = launch_pdl(kernel, dim3(grid), dim3(512), smem, stream, mq, mk, mv, mo, p);
+    const cudaError_t err = launch_pdl(kernel, dim3(grid), dim3(threads), smem, stream, mq, mk, mv, mo, p);
     tm.done();
     return err;
   };
   cudaError_t e;
-  if (o_hp == nullptr) {
-    using L = fa::FwdLayout<D, false>;
-    static std::atomic<uint64_t> attr{0};
-    if (!ensure_smem(fa::fa_fwd_kernel<D, false>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
-    e = launch(fa::fa_fwd_kernel<D, false>, L::SMEM_BYTES, L::NT);
+  if (D == 64) {
+    // column-split kernel: one Q tile per item, two CTAs per SM (one with o_hp)
+    if (o_hp == nullptr) {
+      using L = fa::FwdSplitLayout<64, false>;
+      static std::atomic<uint64_t> attr{0};
+      if (!ensure_smem(fa::fa_fwd_split_kernel<64, false>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
+      e = launch(fa::fa_fwd_split_kernel<64, false>, L::SMEM_BYTES, 1, L::CTAS_PER_SM, L::THREADS);
+    } else {
+      using L = fa::FwdSplitLayout<64, true>;
+      static std::atomic<uint64_t> attr{0};
+      if (!ensure_smem(fa::fa_fwd_split_kernel<64, true>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
+      e = launch(fa::fa_fwd_split_kernel<64, true>, L::SMEM_BYTES, 1, L::CTAS_PER_SM, L::THREADS);
+    }
   } else {
-    using L = fa::FwdLayout<D, true>;
-    static std::atomic<uint64_t> attr{0};
-    if (!ensure_smem(fa::fa_fwd_kernel<D, true>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
-    e = launch(fa::fa_fwd_kernel<D, true>, L::SMEM_BYTES, L::NT);
+    // pair kernel: FwdLayout::NT Q tiles per item, one CTA per SM
+    if (o_hp == nullptr) {
+      using L = fa::FwdLayout<128, false>;
+      static std::atomic<uint64_t> attr{0};
+      if (!ensure_smem(fa::fa_fwd_kernel<128, false>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
+      e = launch(fa::fa_fwd_kernel<128, false>, L::SMEM_BYTES, L::NT, 1, L::THREADS);
+    } else {
+      using L = fa::FwdLayout<128, true>;
+      static std::atomic<uint64_t> attr{0};
+      if (!ensure_smem(fa::fa_fwd_kernel<128, true>, L::SMEM_BYTES, attr)) return FA_ERR_CUDA;
+      e = launch(fa::fa_fwd_kernel<128, true>, L::SMEM_BYTES, L::NT, 1, L::THREADS);
+    }
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : cuda_fail("fa_fwd_kernel launch", e);
@@ -272,15 +290,13 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   }
   const long long rows = static_cast<long long>(BH) * N;
   const int n_blk = (N + 127) / 128;
-  // workspace: delta | fp32 dQ accumulator | per-(bh, query block) counters
+  // workspace: delta | fp32 dQ accumulator | work-item counter (d = 128)
   float* delta = reinterpret_cast<float*>(ws);
   const size_t acc_off = round256(static_cast<size_t>(rows) * 4);
   const size_t acc_bytes = static_cast<size_t>(rows) * D * 4;  // a multiple of 256
   float* dq_acc = reinterpret_cast<float*>(ws + acc_off);
-  unsigned int* dq_cnt = reinterpret_cast<unsigned int*>(ws + acc_off + acc_bytes);
-  unsigned int* item_ctr = dq_cnt + static_cast<size_t>(BH) * n_blk;  // after the per-block counters
-  const long long clear_bytes =
-      static_cast<long long>(acc_bytes + round256((static_cast<size_t>(BH) * n_blk + 1) * 4));
+  unsigned int* item_ctr = reinterpret_cast<unsigned int*>(ws + acc_off + acc_bytes);
+  const long long clear_bytes = static_cast<long long>(acc_bytes) + 256;
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D) ||
       !make_map(&mdo, dO, BH, N, D))
@@ -306,7 +322,6 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.row_m = row_m;
     p.delta = delta;
     p.dq_acc = dq_acc;
-    p.dq_cnt = dq_cnt;
     p.item_ctr = item_ctr;
     // d = 128 item order: heads in groups whose fp32 dQ rows (N * D * 4 bytes
     // per head) fit in 32 MB, a quarter of L2, so the reduce-adds of the items
@@ -318,7 +333,6 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       if (hg > BH) hg = BH;
       p.head_group = static_cast<int>(hg);
     }
-    p.dq = static_cast<__nv_bfloat16*>(dq);
     p.dk = static_cast<__nv_bfloat16*>(dk);
     p.dv = static_cast<__nv_bfloat16*>(dv);
     p.BH = BH;
@@ -353,8 +367,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
     }
   }
-  if (D == 128) {
-    // (at d = 64 the main kernel converts each dQ block once it is complete)
+  {
     const long long n8 = rows * D / 8;
     LaunchTimer tm(FA_KERNEL_BWD_DQ, stream);
     cudaError_t e = launch_pdl(fa::fa_bwd_dq_convert_kernel, dim3(grid_for(n8, 256 * 4)), dim3(256), 0, stream,
@@ -395,8 +408,7 @@ size_t fa_bwd_workspace_dq_offset(int B, int H, int N, int d) {
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (!shape_ok(B, H, N, d) || (d != 64 && d != 128)) return 0;
   const size_t rows = static_cast<size_t>(B) * H * N;
-  const size_t blocks = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128);
-  return round256(rows * 4) + round256(rows * static_cast<size_t>(d) * 4) + round256((blocks + 1) * 4);
+  return round256(rows * 4) + round256(rows * static_cast<size_t>(d) * 4) + 256;
 }
 
 }  // extern "C"

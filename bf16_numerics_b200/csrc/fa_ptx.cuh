@@ -331,13 +331,6 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // wait until every committed bulk group has completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// wait until at most N committed bulk groups are still in flight (complete,
-// not only read)
-template <int N>
-__device__ __forceinline__ void bulk_wait_allow() { asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory"); }
-// async-proxy writes to global memory (completed bulk operations) -> ordered
-// before this thread's later generic-proxy accesses and fences
-__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 // wait until at most one committed bulk group is still in flight
 __device__ __forceinline__ void bulk_wait_all_but_one() { asm volatile("cp.async.bulk.wait_group 1;" ::: "memory"); }
 }  // namespace fa

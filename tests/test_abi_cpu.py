@@ -126,14 +126,14 @@ def test_o_hp_entry_points_argument_errors(lib):
 
 
 def test_workspace_layout(lib):
-    # delta | fp32 dQ accumulator | one uint32 counter per (b, h, 128-row query block) + an item counter
+    # delta | fp32 dQ accumulator | 256 bytes holding the work-item counter of the d = 128 kernel
     B, H, N, d = 8, 12, 1024, 64
     rows = B * H * N
     r256 = lambda x: (x + 255) // 256 * 256
-    assert lib.fa_bwd_workspace_bytes(B, H, N, d) == r256(rows * 4) + r256(rows * d * 4) + r256((B * H * 8 + 1) * 4)
+    assert lib.fa_bwd_workspace_bytes(B, H, N, d) == r256(rows * 4) + r256(rows * d * 4) + 256
     assert lib.fa_bwd_workspace_delta_offset(B, H, N, d) == 0
     assert lib.fa_bwd_workspace_dq_offset(B, H, N, d) == r256(rows * 4)
-    assert lib.fa_bwd_workspace_bytes(1, 1, 100, 128) == r256(400) + r256(100 * 128 * 4) + r256(2 * 4)
+    assert lib.fa_bwd_workspace_bytes(1, 1, 100, 128) == r256(400) + r256(100 * 128 * 4) + 256
     assert lib.fa_bwd_workspace_bytes(1, 1, 128, 96) == 0
 
 
