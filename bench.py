@@ -40,6 +40,7 @@ METRIC = "attention fwd+bwd TFLOP/s (causal) and % of B200 dense BF16 peak, stab
 WORKLOAD = "g2s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ("bf16_numerics_b200/csrc/fa_ptx.cuh", "bf16_numerics_b200/csrc/fa_fwd.cuh",
+                  "bf16_numerics_b200/csrc/fa_fwd_split.cuh",
                   "bf16_numerics_b200/csrc/fa_bwd.cuh", "bf16_numerics_b200/csrc/fa_bwd_pipe.cuh",
                   "bf16_numerics_b200/csrc/fa_bwd_pipe128.cuh", "bf16_numerics_b200/csrc/fa_lib.cu")
 
@@ -219,7 +220,7 @@ def launched_kernel_name(slot: str, d: int) -> str:
     if slot == "fa_bwd_main_kernel":
         return "fa_bwd_main_pipe_kernel" if d == 64 else "fa_bwd_main_pipe128_kernel"
     if slot == "fa_fwd_kernel":
-        return f"fa_fwd_kernel<{d}>"
+        return f"fa_fwd_split_kernel<{d}>" if d == 64 else f"fa_fwd_kernel<{d}>"
     return slot
 
 

@@ -34,8 +34,7 @@ namespace fa {
 
 // ------------------------------------------------------------------ delta
 // delta[r] = sum_c dO[r,c] * O[r,c] in fp32; also clears the dQ accumulator
-// and the work-item counter behind it (with TMA bulk stores of a zeroed
-// shared-memory buffer).  O is the bf16 output of the forward, or (OT = float) its fp32 value
+// rows and the work-item counter behind them.  O is the bf16 output of the forward, or (OT = float) its fp32 value
 // before rounding (the high-precision O_hp of the pages).
 // Memory bound: each row of O and dO is read once with 16-byte loads, LPR
 // lanes per row (8 elements of dO per lane); every warp takes U row groups at
@@ -91,37 +90,18 @@ struct ORaw<float> {
 template <int D, typename OT>
 __global__ void __launch_bounds__(256)
 fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
-                    float* __restrict__ delta, float* __restrict__ dq_acc, long long rows,
-                    long long clear_bytes) {
+                    float* __restrict__ delta, float* __restrict__ dq_acc, long long rows) {
   constexpr int LPR = D / 8;               // lanes per row (8 elements per lane)
   constexpr int RPW = 32 / LPR;            // rows per warp per group
   constexpr int U = 4;                     // row groups per warp per pass
-  constexpr int ZCHUNK = 16384;            // bytes of zeros per bulk store
-  // zeros for the accumulator clear, written by TMA bulk stores so that the
-  // threads' own load/store slots stay with the delta rows
-  __shared__ __align__(128) float4 zeros[ZCHUNK / 16];
   const int lane = threadIdx.x & 31;
   const long long warp_global = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const int sub = lane / LPR, li = lane % LPR;
-  for (int i = threadIdx.x; i < ZCHUNK / 16; i += blockDim.x) zeros[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  fence_proxy_async_smem();
-  __syncthreads();
   grid_launch_dependents();
   grid_dependency_wait();  // O comes from the forward grid; the workspace may be the previous grid's
-  if (threadIdx.x == 0) {
-    // this block's share of the region to clear (the fp32 dQ accumulator and
-    // the work-item counter that follows it; a multiple of 256 bytes):
-    // 16 KB chunks dealt round-robin over the blocks
-    const long long bytes = clear_bytes;
-    const long long nchunk = (bytes + ZCHUNK - 1) / ZCHUNK;
-    for (long long c = blockIdx.x; c < nchunk; c += gridDim.x) {
-      const long long off = c * ZCHUNK;
-      const long long len = bytes - off < ZCHUNK ? bytes - off : ZCHUNK;
-      bulk_store(reinterpret_cast<uint8_t*>(dq_acc) + off, smem_u32(zeros), static_cast<uint32_t>(len));
-    }
-    bulk_commit();
-  }
+  // the 256-byte block after the accumulator (the d = 128 kernel's work-item counter)
+  if (blockIdx.x == 0 && threadIdx.x < 64) reinterpret_cast<unsigned int*>(dq_acc + rows * D)[threadIdx.x] = 0u;
   for (long long r0 = warp_global * (RPW * U); r0 < rows; r0 += n_warps * (RPW * U)) {
     ORaw<OT> a[U];
     uint4 b[U];
@@ -136,6 +116,17 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
         b[u] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
+    // the accumulator rows (plain 16-byte stores measured 12.8 us against 14.9 us
+    // for TMA bulk stores of a zeroed shared buffer on g2s)
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long r = r0 + u * RPW + sub;
+      if (r < rows) {
+        float4* z = reinterpret_cast<float4*>(dq_acc + r * D) + 2 * li;
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       float acc = a[u].dot(b[u], 0.f);
@@ -145,8 +136,6 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
       if (r < rows && li == 0) delta[r] = acc;
     }
   }
-  // the zeros must stay in shared memory until the bulk stores are complete
-  if (threadIdx.x == 0) bulk_wait_all();
 }
 
 // --------------------------------------------------------------- dQ convert

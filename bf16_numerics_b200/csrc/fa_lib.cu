@@ -296,7 +296,6 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   const size_t acc_bytes = static_cast<size_t>(rows) * D * 4;  // a multiple of 256
   float* dq_acc = reinterpret_cast<float*>(ws + acc_off);
   unsigned int* item_ctr = reinterpret_cast<unsigned int*>(ws + acc_off + acc_bytes);
-  const long long clear_bytes = static_cast<long long>(acc_bytes) + 256;
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mk, k, BH, N, D) || !make_map(&mv, v, BH, N, D) ||
       !make_map(&mdo, dO, BH, N, D))
@@ -307,11 +306,10 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     const dim3 grid(grid_for(rows, rows_per_block));
     cudaError_t e =
         o_is_hp ? launch_pdl(fa::fa_bwd_delta_kernel<D, float>, grid, dim3(256), 0, stream,
-                             static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows,
-                             clear_bytes)
+                             static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows)
                 : launch_pdl(fa::fa_bwd_delta_kernel<D, __nv_bfloat16>, grid, dim3(256), 0, stream,
                              static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta,
-                             dq_acc, rows, clear_bytes);
+                             dq_acc, rows);
     tm.done();
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("fa_bwd_delta_kernel launch", e);

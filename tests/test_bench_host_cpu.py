@@ -87,4 +87,5 @@ def test_launched_kernel_names_follow_the_head_dimension():
     assert bench.launched_kernel_name("fa_bwd_main_kernel", 64) == "fa_bwd_main_pipe_kernel"
     assert bench.launched_kernel_name("fa_bwd_main_kernel", 128) == "fa_bwd_main_pipe128_kernel"
     assert bench.launched_kernel_name("fa_fwd_kernel", 128) == "fa_fwd_kernel<128>"
+    assert bench.launched_kernel_name("fa_fwd_kernel", 64) == "fa_fwd_split_kernel<64>"
     assert bench.launched_kernel_name("fa_bwd_delta_kernel", 64) == "fa_bwd_delta_kernel"
