@@ -224,6 +224,26 @@ def launched_kernel_name(slot: str, d: int) -> str:
     return slot
 
 
+def kernel_role(name: str) -> str:
+    """Which step of the path a launched kernel (as launched_kernel_name
+    reports it) performs."""
+    if name.startswith("fa_fwd_"):
+        return "fwd"
+    if name.startswith("fa_bwd_main"):
+        return "bwd_main"
+    if name == "fa_bwd_delta_kernel":
+        return "delta"
+    if name == "fa_bwd_dq_convert_kernel":
+        return "dq_convert"
+    raise ValueError(f"unknown kernel {name}")
+
+
+def kernel_bound(name: str) -> str:
+    """The roofline that bounds a kernel: the forward and the backward main
+    kernels are dense contractions; delta and the dQ conversion stream HBM."""
+    return "tensor" if kernel_role(name) in ("fwd", "bwd_main") else "hbm"
+
+
 def workload_config(w, mode, beta):
     what, inputs = WORKLOAD_TEXT.get(w.name, (w.name, "seeded synthetic"))
     return {"workload": f"{w.name}: {what} B{w.B} H{w.H} N{w.N} d{w.d} {'causal' if w.causal else 'non-causal'}, "
@@ -438,18 +458,13 @@ def run_ours(args, rank, world, local_rank):
         if n_l == 0:
             continue
         avg_s = ms / n_l * 1e-3
-        if name.startswith("fa_fwd_kernel"):
-            kern[name] = {"bound": "tensor", "avg_us": avg_s * 1e6, "achieved": fwd_flops / avg_s / 1e12,
-                          "unit": "TFLOP/s", "frac": fwd_flops / avg_s / 1e12 / peak_tf}
-        elif name.startswith("fa_bwd_main"):
-            kern[name] = {"bound": "tensor", "avg_us": avg_s * 1e6, "achieved": bwd_flops / avg_s / 1e12,
-                          "unit": "TFLOP/s", "frac": bwd_flops / avg_s / 1e12 / peak_tf}
-        elif name == "fa_bwd_delta_kernel":
-            kern[name] = {"bound": "hbm", "avg_us": avg_s * 1e6, "achieved": delta_bytes / avg_s / 1e9,
-                          "unit": "GB/s", "frac": delta_bytes / avg_s / 1e9 / hbm}
+        work = {"fwd": fwd_flops, "bwd_main": bwd_flops, "delta": delta_bytes, "dq_convert": dq_bytes}[kernel_role(name)]
+        if kernel_bound(name) == "tensor":
+            kern[name] = {"bound": "tensor", "avg_us": avg_s * 1e6, "achieved": work / avg_s / 1e12,
+                          "unit": "TFLOP/s", "frac": work / avg_s / 1e12 / peak_tf}
         else:
-            kern[name] = {"bound": "hbm", "avg_us": avg_s * 1e6, "achieved": dq_bytes / avg_s / 1e9,
-                          "unit": "GB/s", "frac": dq_bytes / avg_s / 1e9 / hbm}
+            kern[name] = {"bound": "hbm", "avg_us": avg_s * 1e6, "achieved": work / avg_s / 1e9,
+                          "unit": "GB/s", "frac": work / avg_s / 1e9 / hbm}
         kern[name]["launches"] = n_l
     dominant = max(per_kernel, key=lambda nm: per_kernel[nm][1])
     dk_ = kern[dominant]

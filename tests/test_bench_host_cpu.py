@@ -89,3 +89,13 @@ def test_launched_kernel_names_follow_the_head_dimension():
     assert bench.launched_kernel_name("fa_fwd_kernel", 128) == "fa_fwd_kernel<128>"
     assert bench.launched_kernel_name("fa_fwd_kernel", 64) == "fa_fwd_split_kernel<64>"
     assert bench.launched_kernel_name("fa_bwd_delta_kernel", 64) == "fa_bwd_delta_kernel"
+
+
+def test_every_launched_kernel_has_its_roofline():
+    import bench
+
+    for d in (64, 128):
+        names = [bench.launched_kernel_name(slot, d) for slot in
+                 ("fa_fwd_kernel", "fa_bwd_delta_kernel", "fa_bwd_main_kernel", "fa_bwd_dq_convert_kernel")]
+        assert [bench.kernel_bound(n) for n in names] == ["tensor", "hbm", "tensor", "hbm"]
+        assert [bench.kernel_role(n) for n in names] == ["fwd", "delta", "bwd_main", "dq_convert"]
