@@ -13,6 +13,8 @@
 // The recompute follows the softmax mode:
 //   standard   : P = exp(S - lse)
 //   stabilised : P_bar = exp(S - m), P = P_bar * (1/l), l = exp(lse - m),
+//                (the kernels apply 1/l as the exponent offset -log2(l), so
+//                P = exp2((S - m) log2(e) - (lse - m) log2(e)): one exp2 per score),
 //                with m the row shift the forward selected.
 //
 // Main kernels: a work item is one (batch, head, 128-key block), looping over

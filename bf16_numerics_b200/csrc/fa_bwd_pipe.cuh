@@ -26,7 +26,7 @@
 //     global memory with one TMA tensor reduce-add per 32-column half, one
 //     half after the other through the same box (rows past N are clipped by
 //     the tensor map).  They also prepare the per-query
-//     vectors (lse or m, 1/l, delta) two blocks ahead.
+//     vectors (exponent offset from lse and m, delta) two blocks ahead.
 //
 // Barrier phases count a global query-block index g that runs across the
 // CTA's items; every phase of every barrier is waited for in order and no
@@ -52,8 +52,8 @@ struct BwdPipeLayout {
   static constexpr int DO_OFF = Q_OFF + NST * TILE;
   static constexpr int DS_OFF = DO_OFF + NST * TILE;  // dS^T [keys][queries], two 64-query halves
   static constexpr int DQS_OFF = DS_OFF + 2 * TILE;   // dQ staging: one [128 rows][32 fp32] swizzled box
-  static constexpr int VEC_OFF = DQS_OFF + TILE;      // [2 stages][3][128] fp32
-  static constexpr int BAR_OFF = VEC_OFF + 2 * 3 * 128 * 4;
+  static constexpr int VEC_OFF = DQS_OFF + TILE;      // [2 stages][2][128] fp32
+  static constexpr int BAR_OFF = VEC_OFF + 2 * 2 * 128 * 4;
   enum {
     KV_FULL = 0,
     KV_EMPTY,
@@ -143,7 +143,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   auto bar = [&](int i) { return base + L::BAR_OFF + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
-  // per-query vectors at VEC_OFF, [stage][0]: -a, [stage][1]: 1/l, [stage][2]: delta (fp32 x 128)
+  // per-query vectors at VEC_OFF, [stage][0]: exponent offset, [stage][1]: delta (fp32 x 128)
   const uint64_t limit_ns = wait_limit_ns();
   const BoundedWait wait{abort_flag, 3u, limit_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -365,20 +365,16 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     };
     auto publish_vec = [&](int g, const BwdCursor& c, const Vec3& v) {
       const int s = g & 1, q = c.qblk() * L::B + t;
-      float na = -INFINITY, bb = 0.f, dl = 0.f;
+      float na = -INFINITY, dl = 0.f;
       if (q < p.N) {
         dl = v.dl;
-        if (p.mode == 1) {
-          na = -v.m * kLog2e;
-          bb = 1.f / ex2_approx((v.lse - v.m) * kLog2e);
-        } else {
-          na = -v.lse * kLog2e;
-          bb = 1.f;
-        }
+        // standard: P = exp(S - lse).  Stabilised: P = P_bar / l with
+        // P_bar = exp(S - m) and l = exp(lse - m); the factor 1/l enters as
+        // the exponent offset -log2(l) = -(lse - m) log2(e)
+        na = (p.mode == 1) ? (-v.m * kLog2e - (v.lse - v.m) * kLog2e) : -v.lse * kLog2e;
       }
-      sts32(base + L::VEC_OFF + ((s * 3 + 0) * 128 + t) * 4, na);
-      sts32(base + L::VEC_OFF + ((s * 3 + 1) * 128 + t) * 4, bb);
-      sts32(base + L::VEC_OFF + ((s * 3 + 2) * 128 + t) * 4, dl);
+      sts32(base + L::VEC_OFF + ((s * 2 + 0) * 128 + t) * 4, na);
+      sts32(base + L::VEC_OFF + ((s * 2 + 1) * 128 + t) * 4, dl);
       mbar_arrive(bar(L::VEC_FULL + s));
     };
     // pub walks two blocks ahead of cur, nxt holds the loads for pub
@@ -459,7 +455,6 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     const float scale = p.scale;
     const float c_log2 = scale * kLog2e;
     const uint64_t C2 = f2_pack(c_log2, c_log2);
-    const bool mode1 = p.mode == 1;
     const int qoff = 64 * h;
     const uint32_t ds_row = base + L::DS_OFF + h * TILE + t * 128;
     BwdCursor cur;
@@ -481,9 +476,8 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         ok = ok && wait.warp(bar(L::S_FULL + b), (g >> 1) & 1, 9);
         if (threadIdx.x == 0) FA_TRACE_POINT(20);
         tc_fence_after();
-        const uint32_t va = base + L::VEC_OFF + ((b * 3 + 0) * 128 + 64 * h) * 4;
-        const uint32_t vb = base + L::VEC_OFF + ((b * 3 + 1) * 128 + 64 * h) * 4;
-        const uint32_t vd = base + L::VEC_OFF + ((b * 3 + 2) * 128 + 64 * h) * 4;
+        const uint32_t va = base + L::VEC_OFF + ((b * 2 + 0) * 128 + 64 * h) * 4;
+        const uint32_t vd = base + L::VEC_OFF + ((b * 2 + 1) * 128 + 64 * h) * 4;
         const bool diag = p.causal && (cur.i0 + i == cur.kblk);
         uint64_t p2[32];  // this row's 64 P values (fp32 pairs)
         {
@@ -509,13 +503,13 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           float a0, a1, a2, a3;
           f2_unpack(y0, a0, a1);
           f2_unpack(y1, a2, a3);
-          float p0 = ex2_approx(a0), p1 = ex2_approx(a1), p2v = ex2_approx(a2), p3 = ex2_approx(a3);
-          if (mode1) {
-            const float4 bb = lds128(vb + ql * 4);
-            p0 *= bb.x;
-            p1 *= bb.y;
-            p2v *= bb.z;
-            p3 *= bb.w;
+          float p0 = ex2_approx(a0), p1 = ex2_approx(a1), p2v, p3;
+          if ((pi >> 1) % 4 == 3) {
+            // one pair in eight on the FMA pipe
+            f2_unpack(exp2_poly_f2(y1), p2v, p3);
+          } else {
+            p2v = ex2_approx(a2);
+            p3 = ex2_approx(a3);
           }
           if (diag) {
             const int qg = qoff + ql;

@@ -23,7 +23,7 @@
 //     first half of the dP^T columns each warpgroup has just read
 //     (64h + [0,32)), which needs no barrier, and as a 128B-swizzled tile into
 //     shared memory for dQ.
-//   * Each warpgroup publishes the per-query vectors (exponent offset, 1/l,
+//   * Each warpgroup publishes the per-query vectors (exponent offset,
 //     delta) of its 64 query columns in shared memory at the top of a block,
 //     from values loaded one block ahead.
 //   * Four drain warps add the dQ partial (times the softmax scale) to the
@@ -59,8 +59,8 @@ struct BwdPipe128Layout {
   static constexpr int K_OFF = 0, V_OFF = TILE, Q_OFF = 2 * TILE;
   static constexpr int DO_OFF = Q_OFF + NST * TILE;
   static constexpr int DS_OFF = DO_OFF + NST * TILE;     // dS^T [keys][queries], two 64-query halves
-  static constexpr int VEC_OFF = DS_OFF + TILE;          // [3][128] fp32: exponent offset, 1/l, delta
-  static constexpr int RING_OFF = VEC_OFF + 3 * 128 * 4; // [RING] item numbers (-1: end of the list)
+  static constexpr int VEC_OFF = DS_OFF + TILE;          // [2][128] fp32: exponent offset, delta
+  static constexpr int RING_OFF = VEC_OFF + 2 * 128 * 4; // [RING] item numbers (-1: end of the list)
   static constexpr int RING = 4;
   // threads that read each ring slot: the MMA thread, the 128 drain threads
   // and the 256 elementwise threads twice (their block cursor and the cursor
@@ -469,10 +469,9 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
     const int qoff = 64 * h;
     const uint32_t ds_row = base + L::DS_OFF + h * HALF + t * 128;
     const uint32_t va = base + L::VEC_OFF + (0 * 128 + qoff) * 4;
-    const uint32_t vb = base + L::VEC_OFF + (1 * 128 + qoff) * 4;
-    const uint32_t vd = base + L::VEC_OFF + (2 * 128 + qoff) * 4;
+    const uint32_t vd = base + L::VEC_OFF + (1 * 128 + qoff) * 4;
     // Per-query vectors: thread t publishes query 64h + (t & 63) of the block,
-    // threads t < 64 the exponent offset and 1/l, threads t >= 64 delta.  The
+    // threads t < 64 the exponent offset, threads t >= 64 delta.  The
     // raw values are loaded one block ahead (cursor pf).
     const int vq = t & 63, vrole = t >> 6;
     RingCursor pf{wait, base + L::RING_OFF, bar(L::ITEM_FULL), bar(L::ITEM_EMPTY), true, p};
@@ -512,19 +511,18 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
         // this warpgroup has finished with the previous block's vectors
         named_barrier_sync(3 + h, 128);
         if (vrole == 0) {
-          float na, bb;
+          // standard: P = exp(S - lse).  Stabilised: P = P_bar / l with
+          // P_bar = exp(S - m) and l = exp(lse - m); the factor 1/l enters as
+          // the exponent offset -log2(l) = -(lse - m) log2(e)
+          float na;
           if (nx == INFINITY) {
             na = -INFINITY;
-            bb = 0.f;
           } else if (mode1) {
-            na = -ny * kLog2e;
-            bb = 1.f / ex2_approx((nx - ny) * kLog2e);
+            na = -ny * kLog2e - (nx - ny) * kLog2e;
           } else {
             na = -nx * kLog2e;
-            bb = 1.f;
           }
           sts32(va + vq * 4, na);
-          sts32(vb + vq * 4, bb);
         } else {
           sts32(vd + vq * 4, nx == INFINITY ? 0.f : nx);
         }
@@ -555,13 +553,13 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
           float a0, a1, a2, a3;
           f2_unpack(y0, a0, a1);
           f2_unpack(y1, a2, a3);
-          float p0 = ex2_approx(a0), p1 = ex2_approx(a1), p2v = ex2_approx(a2), p3 = ex2_approx(a3);
-          if (mode1) {
-            const float4 bb = lds128(vb + ql * 4);
-            p0 *= bb.x;
-            p1 *= bb.y;
-            p2v *= bb.z;
-            p3 *= bb.w;
+          float p0 = ex2_approx(a0), p1 = ex2_approx(a1), p2v, p3;
+          if ((pi >> 1) % 4 == 3) {
+            // one pair in eight on the FMA pipe
+            f2_unpack(exp2_poly_f2(y1), p2v, p3);
+          } else {
+            p2v = ex2_approx(a2);
+            p3 = ex2_approx(a3);
           }
           if (diag) {
             const int qg = qoff + ql;

@@ -203,42 +203,65 @@ fa_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         bulk_commit();
         return true;
       };
-      int n = 0, gt = 0;
-      bool ok = true;
-      for (; cur.valid; cur.next(p), ++n) {
-        const int qs = n & 1;
-        if (n >= 2) {
-          // item n-2's O is staged in this buffer: store it, and reuse the
+      // Loads go in the order in which the MMA warp consumes them: K of the
+      // next tile (this item's next one, or the next item's first, followed
+      // there by the next item's Q) ahead of V of the current tile.  A K load
+      // then waits only for the Q K^T two tiles back; loading V(j) before
+      // K(j+1) tied each K load to the P V product two tiles back, and the
+      // softmax warps waited ~600 cycles per tile for their next S.
+      auto load_q = [&](const FwdSplitCursor& c, int m) -> bool {
+        const int qs = m & 1;
+        if (m >= 2) {
+          // item m-2's O is staged in this buffer: store it, and reuse the
           // buffer once the store has read it
-          if (!store_staged(n - 2)) { ok = false; break; }
+          if (!store_staged(m - 2)) return false;
           bulk_wait_read_all();
         }
         mbar_expect_tx(bar(L::Q_FULL + qs), L::TILE);
         for (int hh = 0; hh < D / 64; ++hh)
           tma_load_3d(base + L::Q_OFF + qs * L::TILE + hh * L::HALF, &tm_q, bar(L::Q_FULL + qs), 64 * hh,
-                      cur.qblk * L::BM, cur.bh);
-        q_issued = n + 1;
-        for (int j = 0; j < cur.nkv; ++j, ++gt) {
-          const int s = gt & 1, u = gt >> 1;
-          if (u > 0 && !wait(bar(L::K_EMPTY + s), (u - 1) & 1, 2)) { ok = false; break; }
-          mbar_expect_tx(bar(L::K_FULL + s), L::TILE);
-          for (int hh = 0; hh < D / 64; ++hh)
-            tma_load_3d(base + L::K_OFF + s * L::TILE + hh * L::HALF, &tm_k, bar(L::K_FULL + s), 64 * hh,
-                        j * L::BN, cur.bh);
-          k_issued = gt + 1;
-          if (gt == 0) {
-            // cold start: let the first Q K^T's operands arrive before the
-            // rest of the rings competes with them for DRAM
-            if (!wait(bar(L::Q_FULL), 0, 23) || !wait(bar(L::K_FULL), 0, 24)) { ok = false; break; }
+                      c.qblk * L::BM, c.bh);
+        q_issued = m + 1;
+        return true;
+      };
+      auto load_k = [&](const FwdSplitCursor& c, int j, int g) -> bool {
+        const int s = g & 1, u = g >> 1;
+        if (u > 0 && !wait(bar(L::K_EMPTY + s), (u - 1) & 1, 2)) return false;
+        mbar_expect_tx(bar(L::K_FULL + s), L::TILE);
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_3d(base + L::K_OFF + s * L::TILE + hh * L::HALF, &tm_k, bar(L::K_FULL + s), 64 * hh,
+                      j * L::BN, c.bh);
+        k_issued = g + 1;
+        return true;
+      };
+      auto load_v = [&](const FwdSplitCursor& c, int j, int g) -> bool {
+        const int s = g & 1, u = g >> 1;
+        if (u > 0 && !wait(bar(L::V_EMPTY + s), (u - 1) & 1, 3)) return false;
+        mbar_expect_tx(bar(L::V_FULL + s), L::TILE);
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_3d(base + L::V_OFF + s * L::TILE + hh * L::HALF, &tm_v, bar(L::V_FULL + s), 64 * hh,
+                      j * L::BN, c.bh);
+        v_issued = g + 1;
+        return true;
+      };
+      int n = 0, gt = 0;
+      bool ok = true;
+      if (cur.valid) {
+        // cold start: let the first Q K^T's operands arrive before the rest
+        // of the rings competes with them for DRAM
+        ok = load_q(cur, 0) && load_k(cur, 0, 0) && wait(bar(L::Q_FULL), 0, 23) && wait(bar(L::K_FULL), 0, 24);
+      }
+      for (; ok && cur.valid; cur.next(p), ++n) {
+        for (int j = 0; ok && j < cur.nkv; ++j, ++gt) {
+          if (j + 1 < cur.nkv) {
+            ok = load_k(cur, j + 1, gt + 1);
+          } else if (cur.has_next(p)) {
+            FwdSplitCursor nx = cur;
+            nx.next(p);
+            ok = load_k(nx, 0, gt + 1) && load_q(nx, n + 1);
           }
-          if (u > 0 && !wait(bar(L::V_EMPTY + s), (u - 1) & 1, 3)) { ok = false; break; }
-          mbar_expect_tx(bar(L::V_FULL + s), L::TILE);
-          for (int hh = 0; hh < D / 64; ++hh)
-            tma_load_3d(base + L::V_OFF + s * L::TILE + hh * L::HALF, &tm_v, bar(L::V_FULL + s), 64 * hh,
-                        j * L::BN, cur.bh);
-          v_issued = gt + 1;
+          ok = ok && load_v(cur, j, gt);
         }
-        if (!ok) break;
       }
       // the O tiles still staged: the last two items
       if (ok) {
