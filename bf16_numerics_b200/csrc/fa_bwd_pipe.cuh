@@ -297,7 +297,8 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           // dV += P^T dO_g   (K-dim = queries; P^T at S^T cols [0,64))
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ts(tmem + L::DV_COL, tmem + 128u * b + 8u * ks, sdesc_sw128(do_tile(g) + ks * 2048, 16384, 1024),
+            mma_ts(tmem + L::DV_COL, tmem + 128u * b + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4)),
+                   sdesc_sw128(do_tile(g) + ks * 2048, 16384, 1024),
                    IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
           if (!wait(bar(L::DS_FULL), g & 1, 5)) { ok = false; break; }
           FA_TRACE_POINT(11);
@@ -460,16 +461,16 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     BwdCursor cur;
     cur.start(p);
     int g = 0;
-    // Error discipline: the two warpgroups meet on named barrier 1 once per
-    // block and once per item.  A bounded wait that gives up only clears `ok`
-    // (reads before the next meeting may see stale TMEM or shared memory,
-    // which is in bounds and harmless); each meeting is an AND vote, so both
-    // warpgroups leave together and neither is left waiting on a barrier the
-    // other no longer reaches.
+    // Error discipline: the eight warps meet on named barrier 1 once per item,
+    // at the AND vote of the item's epilogue (each warpgroup writes its P^T
+    // over its own S^T columns, so they need no meeting per block).  A bounded
+    // wait that gives up only clears `ok`; the warp then goes on to the
+    // epilogue (its reads there may see stale TMEM or shared memory, which is
+    // in bounds and harmless), so every warp reaches the vote and all leave
+    // together.
     bool ok = true;
     const bool stall = inject_stall_here(3u);  // test hook (fa_debug_inject_stall)
     for (; cur.valid; cur.next_item()) {
-      bool leave = false;
       for (int i = 0; i < cur.n; ++i, ++g) {
         const int b = g & 1;
         ok = ok && wait.warp(bar(L::VEC_FULL + b), (g >> 1) & 1, 8);
@@ -491,7 +492,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         }
         if (threadIdx.x == 0) FA_TRACE_POINT(25);
         // both warpgroups hold their S^T columns: P^T may now overwrite [0,64)
-        if (!named_barrier_and(1, 256, ok)) { leave = true; break; }
+        if (!ok) break;  // to the item's epilogue and its vote
         if (threadIdx.x == 0) FA_TRACE_POINT(26);
         uint32_t pk[32];
 #pragma unroll
@@ -523,7 +524,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           pk[pi] = pack_bf16x2(p0, p1);
           pk[pi + 1] = pack_bf16x2(p2v, p3);
         }
-        tmem_st32(tmem + lane_base + 128u * b + 32u * h, pk);
+        tmem_st32(tmem + lane_base + 128u * b + 64u * h, pk);
         if (threadIdx.x == 0) FA_TRACE_POINT(27);
         tmem_st_wait();
         tc_fence_before();
@@ -572,7 +573,11 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         mbar_arrive(bar(L::VEC_EMPTY + b));
         if (threadIdx.x == 0) FA_TRACE_POINT(24);
       }
-      if (leave) break;
+      // A warp that gave up on a wait (ok false) still takes the
+      // epilogue below: its reads there are stale but in bounds, and the AND
+      // vote on named barrier 1 is the meeting that takes all eight warps out
+      // together (the warpgroups do not meet per block, so another warp may
+      // already be waiting at that vote).
       // ----------------------------------------------------- item epilogue
       // warpgroup 0 writes dV, warpgroup 1 writes dK * scale: TMEM -> bf16
       // rows in a 128B-swizzled tile (its half of the dS tile, whose last
