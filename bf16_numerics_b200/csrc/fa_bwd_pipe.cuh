@@ -13,14 +13,15 @@
 //     g+2 while the elementwise warps work on block g, and dP^T of block g+1
 //     as soon as block g's dS has been consumed.
 //   * Eight elementwise warps (two warpgroups) split the 128 query columns of
-//     a key row: warpgroup h takes columns [64h, 64h+64).  Both copy their S^T
-//     columns to registers and meet at a named barrier; then warpgroup h
-//     writes its bf16 P^T into S^T cols [32h, 32h+32), so P^T occupies
-//     [0,64) and [64,128) is free for dQ.  dS^T goes into the first half of
-//     the dP^T columns each warpgroup has just read (64h + [0,32)), which
-//     needs no barrier.
+//     a key row: warpgroup h takes columns [64h, 64h+64).  Each copies its
+//     S^T columns to registers and writes its bf16 P^T over the first half of
+//     them (64h + [0,32)), so the warpgroups never touch each other's columns
+//     and need no meeting per block; the dV product reads P^T at [0,32) and
+//     [64,96).  dS^T goes into the first half of the dP^T columns each
+//     warpgroup has just read (64h + [0,32)).
 //   * dQ_g = dS K is one N = 64 product into S^T cols [64,128) of the same
-//     buffer, which no later product of the block touches.
+//     buffer, issued after dV_g has read P^T there (products from one thread
+//     run in issue order); no later product of the block touches it.
 //   * Four drain warps move the dQ partial from TMEM into a 128B-swizzled
 //     fp32 staging box in shared memory and add it to the fp32 accumulator in
 //     global memory with one TMA tensor reduce-add per 32-column half, one
@@ -294,7 +295,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           // previous item's epilogue must have copied them out
           if (i == 0 && cur.r > 0 && !wait(bar(L::ACC_FREE), (cur.r - 1) & 1, 8)) { ok = false; break; }
           tc_fence_after();
-          // dV += P^T dO_g   (K-dim = queries; P^T at S^T cols [0,64))
+          // dV += P^T dO_g   (K-dim = queries; P^T at S^T cols [0,32) and [64,96))
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
             mma_ts(tmem + L::DV_COL, tmem + 128u * b + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4)),
