@@ -86,7 +86,7 @@ def test_two_hot_ties_against_the_bf16_ds_reference(cuda_device, causal, N):
     opposite terms (dS[t,0] + dS[t,j*]) K[0]; rounding dS to BF16 -- the
     operand precision of the dQ product -- moves it by up to about 2 % of
     max|dQ| (tests/test_oracle_attention.py: the floor exceeds 1e-2 on such
-    rows).  dQ and dK meet the spec bar against the oracle with that
+    rows).  dQ and dK meet the 1e-2 bar against the oracle with that
     operand modelled; O and dV against the float64 oracle."""
     w = _d128_case(N, causal, 0.5)
     mode = 1
@@ -310,7 +310,7 @@ def test_o_hp_backward_removes_the_delta_bias(cuda_device, name):
 @pytest.mark.parametrize("name", ["tiestress", "g2s", "long"])
 def test_o_hp_pair_meets_the_bar_end_to_end(cuda_device, name):
     """End to end against the chained float64 oracle (delta from the exact O):
-    fa_fwd_o_hp -> fa_bwd_o_hp at full size meets the spec bar on O,
+    fa_fwd_o_hp -> fa_bwd_o_hp at full size meets the 1e-2 bar on O,
     dQ, dK and dV of sampled heads.  (The default fa_fwd -> fa_bwd pair carries
     the delta bias of its bf16 O and misses it on the tie-stress dQ; see
     test_o_hp_backward_removes_the_delta_bias.)"""
