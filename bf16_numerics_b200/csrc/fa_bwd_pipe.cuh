@@ -506,22 +506,20 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         const uint32_t vd = base + L::VEC_OFF + ((b * 2 + 1) * 128 + 64 * h) * 4;
         const bool diag = p.causal && (cur.i0 + i == cur.kblk);
         uint64_t p2[32];  // this row's 64 P values (fp32 pairs)
+        uint32_t rs1[32];  // S^T columns 32-63, loading while the first half is computed
         {
-          uint32_t r0[32], r1[32];
-          tmem_ld32x2(tmem + lane_base + 128u * b + 64u * h, tmem + lane_base + 128u * b + 64u * h + 32u, r0, r1);
+          uint32_t r0[32];
+          tmem_ld32(tmem + lane_base + 128u * b + 64u * h, r0);
+          tmem_ld32_nowait(tmem + lane_base + 128u * b + 64u * h + 32u, rs1);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            p2[e] = f2_pack(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
-            p2[16 + e] = f2_pack(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
-          }
+          for (int e = 0; e < 16; ++e) p2[e] = f2_pack(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
         }
         if (threadIdx.x == 0) FA_TRACE_POINT(25);
         // both warpgroups hold their S^T columns: P^T may now overwrite [0,64)
         if (!ok) break;  // to the item's epilogue and its vote
         if (threadIdx.x == 0) FA_TRACE_POINT(26);
         uint32_t pk[32];
-#pragma unroll
-        for (int pi = 0; pi < 32; pi += 2) {
+        auto p_pair = [&](int pi) {
           const int ql = 2 * pi;
           const float4 na = lds128(va + ql * 4);
           const uint64_t y0 = f2_fma(p2[pi], C2, f2_pack(na.x, na.y));
@@ -548,7 +546,14 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           p2[pi + 1] = f2_pack(p2v, p3);
           pk[pi] = pack_bf16x2(p0, p1);
           pk[pi + 1] = pack_bf16x2(p2v, p3);
-        }
+        };
+#pragma unroll
+        for (int pi = 0; pi < 16; pi += 2) p_pair(pi);
+        tmem_wait_ld32(rs1);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) p2[16 + e] = f2_pack(__uint_as_float(rs1[2 * e]), __uint_as_float(rs1[2 * e + 1]));
+#pragma unroll
+        for (int pi = 16; pi < 32; pi += 2) p_pair(pi);
         tmem_st32(tmem + lane_base + 128u * b + 64u * h, pk);
         if (threadIdx.x == 0) FA_TRACE_POINT(27);
         tmem_st_wait();
@@ -562,15 +567,12 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (!ok) continue;  // the next meeting takes everyone out
         tc_fence_after();
         uint32_t dpr[64];
-        {
-          uint32_t(&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]);
-          uint32_t(&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]);
-          tmem_ld32x2(tmem + lane_base + L::DPT_COL + 64u * h, tmem + lane_base + L::DPT_COL + 64u * h + 32u, d0,
-                      d1);
-        }
+        uint32_t(&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]);
+        uint32_t(&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]);
+        tmem_ld32(tmem + lane_base + L::DPT_COL + 64u * h, d0);
+        tmem_ld32_nowait(tmem + lane_base + L::DPT_COL + 64u * h + 32u, d1);  // in flight during the first half
         uint32_t dk_[32];
-#pragma unroll
-        for (int pi = 0; pi < 32; pi += 2) {
+        auto ds_pair = [&](int pi) {
           const int ql = 2 * pi;
           const float4 dl = lds128(vd + ql * 4);
           const uint64_t ds0 = f2_mul(
@@ -583,7 +585,12 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           f2_unpack(ds1, d2, d3);
           dk_[pi] = pack_bf16x2(d0, d1);
           dk_[pi + 1] = pack_bf16x2(d2, d3);
-        }
+        };
+#pragma unroll
+        for (int pi = 0; pi < 16; pi += 2) ds_pair(pi);
+        tmem_wait_ld32(d1);
+#pragma unroll
+        for (int pi = 16; pi < 32; pi += 2) ds_pair(pi);
         // dS^T into the dP^T columns this warpgroup has read: 64h + [0,32)
         tmem_st32(tmem + lane_base + L::DPT_COL + 64u * h, dk_);
         // dS^T row t, queries 64h + [0,64) = the eight 16-byte chunks of the half tile's row

@@ -252,6 +252,11 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
 }
 #define FA_U8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
+// wait for every outstanding tcgen05.ld; r (32 registers a no-wait load
+// targets) is passed through so that no use of it moves above the wait
+__device__ __forceinline__ void tmem_wait_ld32(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : FA_U8(0), FA_U8(8), FA_U8(16), FA_U8(24));
+}
 __device__ __forceinline__ void tmem_ld32x4(uint32_t taddr, uint32_t (&r)[128]) {
   tmem_ld32_nowait(taddr, &r[0]);
   tmem_ld32_nowait(taddr + 32, &r[32]);
