@@ -410,6 +410,19 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     bool ok = true;
     for (int g = 0; cur.valid; ++g, cur.next_block()) {
       const int b = g & 1;
+      // the vectors of block g+2 first: they are ready once the elementwise
+      // warps have finished block g (VEC_EMPTY), before dQ_g completes
+      if (pub.valid) {
+        // block g+2 reuses the vector stage of block g
+        // (a wait that gives up skips the publish; the next vote ends the loop)
+        ok = wait(bar(L::VEC_EMPTY + b), (g >> 1) & 1, 14) && ok;
+        if (ok) {
+          publish_vec(g_pub, pub, nxt);
+          ++g_pub;
+          pub.next_block();
+          nxt = load_vec(pub);
+        }
+      }
       {
         // every lane calls the warp-uniform wait (ok may differ per lane here)
         const bool got = wait.warp(bar(L::DQ_FULL + b), (g >> 1) & 1, 13);
@@ -448,17 +461,6 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         }
       }
       if (t == 0) FA_TRACE_POINT(31);
-      if (pub.valid) {
-        // block g+2 reuses the vector stage of block g
-        // (a wait that gives up skips the publish; the next vote ends the loop)
-        ok = wait(bar(L::VEC_EMPTY + b), (g >> 1) & 1, 14);
-        if (ok) {
-          publish_vec(g_pub, pub, nxt);
-          ++g_pub;
-          pub.next_block();
-          nxt = load_vec(pub);
-        }
-      }
     }
     if (t == 0) {
       // every reduce-add of this CTA has completed: count it for the dQ
