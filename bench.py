@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark: causal attention fwd+bwd TFLOP/s on B200, stabilised softmax.
 
-One step = fa_fwd + fa_bwd (delta, main; dQ convert at d = 128) on the GPT-2-small
+One step = fa_fwd + fa_bwd (delta, main, dQ convert) on the GPT-2-small
 attention workload (B8 H12 N1024 d64, causal, beta = 2), inputs resident in
 HBM.  The inputs (50 MB) fit in the 126 MB L2, so L2 is flushed (a 256 MiB
 write) before every timed step; the flush is outside the CUDA-event intervals.
@@ -452,7 +452,7 @@ def run_ours(args, rank, world, local_rank):
     bwd_flops = 2.5 * fwd_flops
     rows = B * H * N
     delta_bytes = rows * d * 2 * 2 + rows * 4  # algorithmic: read O, dO; write delta (the dQ clear is overhead)
-    dq_bytes = rows * d * 4 + rows * d * 2  # d = 128 dQ convert: read the fp32 accumulator, write bf16
+    dq_bytes = rows * d * 4 + rows * d * 2  # dQ convert: read the fp32 accumulator, write bf16
     kern = {}
     for name, (n_l, ms) in per_kernel.items():
         if n_l == 0:

@@ -25,7 +25,7 @@ FA_SOFTMAX_STABILIZED_MARGIN = 2
 FA_KERNEL_FWD = 0
 FA_KERNEL_BWD_DELTA = 1
 FA_KERNEL_BWD_MAIN = 2
-FA_KERNEL_BWD_DQ = 3  # d = 128 only (d = 64 converts dQ in the main kernel)
+FA_KERNEL_BWD_DQ = 3
 FA_NUM_KERNELS = 4
 
 # kernel ids in the device error word (fa_device_error) and for fa_debug_inject_stall

@@ -1,7 +1,6 @@
-// Backward kernels: the delta preprocess, the dQ conversion (a kernel of its
-// own at d = 128, the end of the main kernel at d = 64), and the parameters
-// of the dQ/dK/dV main kernels (fa_bwd_pipe.cuh for d = 64,
-// fa_bwd_pipe128.cuh for d = 128).
+// Backward kernels: delta preprocess, dQ convert, and the parameters of the
+// dQ/dK/dV main kernels (fa_bwd_pipe.cuh for d = 64, fa_bwd_pipe128.cuh for
+// d = 128).
 //
 // Gradient of O = softmax(S) V with S = Q K^T * scale (the standard
 // attention backward; the pages name its delta step -- 91haoming.cn page,
@@ -142,8 +141,6 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
 }
 
 // --------------------------------------------------------------- dQ convert
-// Separate conversion kernel (d = 128, whose accumulator is larger than L2:
-// measured faster than converting at the end of the main kernel):
 // dq = bf16(dq_acc), 8 values per thread and chunk, U chunks per thread per
 // pass with all loads issued first; the accumulator is dead afterwards, so
 // it is read with the streaming (evict-first) hint.
@@ -178,42 +175,6 @@ fa_bwd_dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __rest
   }
 }
 
-// dQ conversion inside a persistent main kernel, after every CTA's reduce-adds
-// have completed: this CTA's slice [c n8 / G, (c+1) n8 / G) of the 8-value
-// chunks of the fp32 accumulator -> bf16, by threads [0, T) of the CTA, U
-// chunks per thread per pass with all loads issued first (enough bytes in
-// flight for an accumulator larger than L2).  The accumulator was written by
-// other SMs' reduce-adds, so the loads bypass L1 (.cg).
-template <int U>
-__device__ __forceinline__ void dq_convert_slice(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq,
-                                                 long long n8, int tid, int T) {
-  const long long G = gridDim.x;
-  const long long lo = n8 * blockIdx.x / G, hi = n8 * (blockIdx.x + 1) / G;
-  for (long long i0 = lo + tid; i0 < hi; i0 += static_cast<long long>(T) * U) {
-    float4 a[U], b[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const long long i = i0 + static_cast<long long>(u) * T;
-      if (i < hi) {
-        a[u] = __ldcg(reinterpret_cast<const float4*>(dq_acc) + 2 * i);
-        b[u] = __ldcg(reinterpret_cast<const float4*>(dq_acc) + 2 * i + 1);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const long long i = i0 + static_cast<long long>(u) * T;
-      if (i < hi) {
-        uint4 w;
-        w.x = pack_bf16x2(a[u].x, a[u].y);
-        w.y = pack_bf16x2(a[u].z, a[u].w);
-        w.z = pack_bf16x2(b[u].x, b[u].y);
-        w.w = pack_bf16x2(b[u].z, b[u].w);
-        reinterpret_cast<uint4*>(dq)[i] = w;
-      }
-    }
-  }
-}
-
 // --------------------------------------------------------------- main kernel
 struct BwdParams {
   const float* lse;    // [BH, N]
@@ -222,11 +183,6 @@ struct BwdParams {
   float* dq_acc;       // [BH, N, D] fp32, zeroed by the delta kernel
   unsigned int* item_ctr;  // d = 128: next unclaimed work item (zeroed by the delta kernel)
   int head_group;          // d = 128: heads per group of the item order
-  // d = 64: dQ conversion at the end of the main kernel: every CTA counts its
-  // completed reduce-adds on done_ctr (zeroed by the delta kernel) and, once
-  // all have, converts its slice of the accumulator to bf16 dq
-  unsigned int* done_ctr;
-  __nv_bfloat16* dq;
   __nv_bfloat16* dk;   // [BH, N, D]
   __nv_bfloat16* dv;   // [BH, N, D]
   int BH, N, n_blk;

@@ -199,23 +199,6 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       drain(bar(L::TEARDOWN), 0, 30);
       tmem_dealloc(tmem, L::TMEM_COLS);
     }
-    // dQ: once every CTA's reduce-adds have completed (done_ctr == G), the
-    // elementwise warps (the role with the registers for 16 chunks in flight
-    // per thread) convert this CTA's slice of the accumulator to bf16
-    // (twice the usual limit: the CTAs waited for have bounded waits of their
-    // own, and one that gives up still counts, so the first error recorded is
-    // the wait that caused it)
-    volatile int* conv_go = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
-    if (threadIdx.x == 0) {
-      const volatile unsigned int* dc = p.done_ctr;
-      const BoundedWait final_wait{abort_flag, 3u, 2 * limit_ns};
-      *conv_go = final_wait.until([&] { return *dc >= gridDim.x; }, 29) ? 1 : 0;
-    }
-    named_barrier_sync(14, L::THREADS);
-    if (*conv_go && warp < 8) {
-      __threadfence();
-      dq_convert_slice<16>(p.dq_acc, p.dq, static_cast<long long>(p.BH) * p.N * L::D / 8, threadIdx.x, 256);
-    }
   };
 
   if (warp >= 12) {
@@ -462,14 +445,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       }
       if (t == 0) FA_TRACE_POINT(31);
     }
-    if (t == 0) {
-      // every reduce-add of this CTA has completed: count it for the dQ
-      // conversion of all CTAs (generic loads of other CTAs follow)
-      bulk_wait_all();
-      fence_proxy_async_global();
-      __threadfence();
-      atomicAdd(p.done_ctr, 1u);
-    }
+    if (t == 0) bulk_wait_all();
     teardown();
     return;
   }

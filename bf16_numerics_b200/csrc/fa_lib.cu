@@ -321,8 +321,6 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.delta = delta;
     p.dq_acc = dq_acc;
     p.item_ctr = item_ctr;
-    p.done_ctr = item_ctr + 1;  // zeroed with the rest of the 256-byte block by the delta kernel
-    p.dq = static_cast<__nv_bfloat16*>(dq);
     // d = 128 item order: heads in groups whose fp32 dQ rows (N * D * 4 bytes
     // per head) fit in 32 MB, a quarter of L2, so the reduce-adds of the items
     // in flight hit L2
@@ -367,7 +365,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       if (e != cudaSuccess) return cuda_fail("fa_bwd main kernel launch", e);
     }
   }
-  if (D != 64) {  // d = 64: the main kernel converts dQ itself
+  {
     const long long n8 = rows * D / 8;
     LaunchTimer tm(FA_KERNEL_BWD_DQ, stream);
     cudaError_t e = launch_pdl(fa::fa_bwd_dq_convert_kernel, dim3(grid_for(n8, 256 * 4)), dim3(256), 0, stream,

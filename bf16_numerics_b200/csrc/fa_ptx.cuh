@@ -116,26 +116,6 @@ struct BoundedWait {
   __device__ __forceinline__ bool warp(uint32_t bar, uint32_t parity, uint32_t site) const {
     return __all_sync(0xffffffffu, (*this)(bar, parity, site));
   }
-  // Bounded spin on a condition over global memory that other CTAs update
-  // (pred re-reads it); same time limit, error word and abort flag.
-  template <typename Pred>
-  __device__ __forceinline__ bool until(Pred pred, uint32_t site) const {
-    if (pred()) return true;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
-      __nanosleep(32);
-      if (pred()) return true;
-      if ((it & 63u) == 0u) {
-        if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > limit_ns) {
-          atomicCAS(&g_fa_error, 0u, (kernel_id << 24) | ((site & 0xFFu) << 16) | (blockIdx.x & 0xFFFFu));
-          *abort_flag = 1;
-          __threadfence_block();
-          return false;
-        }
-      }
-    }
-  }
 };
 
 // Named barrier 1 over the first four warps (128 threads).
@@ -157,11 +137,6 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
 // generic-proxy shared-memory writes -> visible to the async proxy (tensor core, TMA)
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-// async-proxy global-memory writes (completed TMA reduce-adds) ordered before
-// the thread's later generic-proxy accesses
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ------------------------------------------------------------------- tcgen05

@@ -100,13 +100,12 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int B, int H, int N, int d, int causal, int softmax_mode, float beta, void* stream);
 
 /* Bytes of device workspace fa_bwd needs: delta (fp32 [B,H,N]), the fp32 dQ
- * accumulator [B,H,N,d] and a 256-byte block that holds two counters of the
- * main kernel (the d = 128 work-item counter, and the count of CTAs whose dQ
- * reduce-adds have completed), each part 256-byte aligned.  0 on bad sizes. */
+ * accumulator [B,H,N,d] and a 256-byte block that holds the work-item counter
+ * of the d = 128 kernel, each part 256-byte aligned.  0 on bad sizes. */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
 /* Byte offset of delta and of the fp32 dQ accumulator inside the workspace
- * (the 256-byte counter block follows the accumulator). */
+ * (the work-item counter follows the accumulator). */
 size_t fa_bwd_workspace_delta_offset(int B, int H, int N, int d);
 size_t fa_bwd_workspace_dq_offset(int B, int H, int N, int d);
 
@@ -114,12 +113,10 @@ size_t fa_bwd_workspace_dq_offset(int B, int H, int N, int d);
  * (fp32 shift m from fa_fwd's stats; required in the stabilised modes,
  * ignored otherwise); outputs dq, dk, dv (bf16).  workspace: caller-owned device
  * memory of at least fa_bwd_workspace_bytes, 256-byte aligned; its contents
- * on entry do not matter and on exit hold delta and the fp32 dQ.  Launches on
- * `stream`: delta (which also clears the accumulator and the counter block),
- * main (dK, dV; dQ accumulated in fp32 by reduce-adds), and the dQ conversion
- * to bf16 -- at d = 64 done by the main kernel itself once every CTA's
- * reduce-adds have completed, at d = 128 a third kernel (FA_KERNEL_BWD_DQ).
- * softmax_mode must match the one the forward used. */
+ * on entry do not matter and on exit hold delta and the fp32 dQ.  Launches
+ * three kernels on `stream`: delta (which also clears the accumulator and the
+ * work-item counter), main (dK, dV, partial dQ), dQ convert.  softmax_mode
+ * must match the one the forward used. */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  const float* row_m, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
                  int H, int N, int d, int causal, int softmax_mode, float beta, void* stream);
