@@ -301,13 +301,13 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       !make_map(&mdo, dO, BH, N, D))
     return cuda_fail("cuTensorMapEncodeTiled (q/k/v/dO)");
   {
-    constexpr int rows_per_block = 8 * (32 / (D / 8)) * 4;  // 8 warps x rows per group x 4 groups
+    constexpr int rows_per_block = 4 * (32 / (D / 8)) * 2;  // 4 warps x rows per group x 2 groups
     LaunchTimer tm(FA_KERNEL_BWD_DELTA, stream);
     const dim3 grid(grid_for(rows, rows_per_block));
     cudaError_t e =
-        o_is_hp ? launch_pdl(fa::fa_bwd_delta_kernel<D, float>, grid, dim3(256), 0, stream,
+        o_is_hp ? launch_pdl(fa::fa_bwd_delta_kernel<D, float>, grid, dim3(128), 0, stream,
                              static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows)
-                : launch_pdl(fa::fa_bwd_delta_kernel<D, __nv_bfloat16>, grid, dim3(256), 0, stream,
+                : launch_pdl(fa::fa_bwd_delta_kernel<D, __nv_bfloat16>, grid, dim3(128), 0, stream,
                              static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta,
                              dq_acc, rows);
     tm.done();
