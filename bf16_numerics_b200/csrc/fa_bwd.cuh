@@ -36,7 +36,7 @@ namespace fa {
 
 // ------------------------------------------------------------------ delta
 // delta[r] = sum_c dO[r,c] * O[r,c] in fp32; also clears the dQ accumulator
-// rows and the work-item counter behind them.  O is the bf16 output of the
+// and the work-item counter behind it.  O is the bf16 output of the
 // forward, or (OT = float) its fp32 value before rounding (the
 // high-precision O_hp of the pages).
 // Memory bound: each row of O and dO is read once with 16-byte loads, LPR
@@ -46,6 +46,13 @@ namespace fa {
 // (two per SM, 80 registers x 384 threads each), so with programmatic
 // dependent launch they are resident when the forward ends (measured: g2s
 // step 123.0 -> 122.4 us, long 2415 -> 2392 us, against 256-thread blocks).
+// The clear does not depend on the forward: every block zeroes its own
+// contiguous share of the accumulator before it waits for the forward grid,
+// so the blocks resident beside the forward's CTAs clear theirs while it
+// runs (measured against clearing each block's rows in the dot loop: g2s
+// step 123.1 -> 121.3 us, long 2396 -> 2373 us).  The one kernel of this
+// library that reads the accumulator, the dQ convert of an earlier call, lets
+// its dependents start only after its last read.
 // 8 consecutive elements of O as they sit in memory (16 bytes of bf16 or
 // 32 bytes of fp32), and their dot product with 8 bf16 elements of dO
 template <typename OT>
@@ -105,9 +112,15 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
   const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const int sub = lane / LPR, li = lane % LPR;
   grid_launch_dependents();
-  grid_dependency_wait();  // O comes from the forward grid; the workspace may be the previous grid's
-  // the 256-byte block after the accumulator (the d = 128 kernel's work-item counter)
-  if (blockIdx.x == 0 && threadIdx.x < 64) reinterpret_cast<unsigned int*>(dq_acc + rows * D)[threadIdx.x] = 0u;
+  {
+    const long long n4 = rows * (D / 4);
+    const long long lo = n4 * blockIdx.x / gridDim.x, hi = n4 * (blockIdx.x + 1) / gridDim.x;
+    float4* acc4 = reinterpret_cast<float4*>(dq_acc);
+    for (long long i = lo + threadIdx.x; i < hi; i += blockDim.x) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    // the 256-byte block after the accumulator (the d = 128 kernel's work-item counter)
+    if (blockIdx.x == 0 && threadIdx.x < 64) reinterpret_cast<unsigned int*>(dq_acc + rows * D)[threadIdx.x] = 0u;
+  }
+  grid_dependency_wait();  // O comes from the forward grid
   for (long long r0 = warp_global * (RPW * U); r0 < rows; r0 += n_warps * (RPW * U)) {
     ORaw<OT> a[U];
     uint4 b[U];
@@ -120,17 +133,6 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
       } else {
         a[u].zero();
         b[u] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-    // the accumulator rows (plain 16-byte stores measured 12.8 us against 14.9 us
-    // for TMA bulk stores of a zeroed shared buffer on g2s)
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const long long r = r0 + u * RPW + sub;
-      if (r < rows) {
-        float4* z = reinterpret_cast<float4*>(dq_acc + r * D) + 2 * li;
-        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
 #pragma unroll
@@ -152,7 +154,6 @@ __global__ void __launch_bounds__(256)
 fa_bwd_dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq, long long n8) {
   constexpr int U = 4;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  grid_launch_dependents();
   grid_dependency_wait();  // the accumulator is complete once the main grid is
   for (long long i0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < n8; i0 += stride * U) {
     float4 a[U], b[U];
@@ -177,6 +178,10 @@ fa_bwd_dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __rest
       }
     }
   }
+  // the delta kernel of a later call clears the accumulator before its own
+  // dependency wait: let it start only once every read here has been used
+  __syncthreads();
+  grid_launch_dependents();
 }
 
 // --------------------------------------------------------------- main kernel
