@@ -50,7 +50,9 @@ namespace fa {
 // contiguous share of the accumulator before it waits for the forward grid,
 // so the blocks resident beside the forward's CTAs clear theirs while it
 // runs (measured against clearing each block's rows in the dot loop: g2s
-// step 123.1 -> 121.3 us, long 2396 -> 2373 us).  The one kernel of this
+// step 123.1 -> 121.3 us, long 2396 -> 2373 us).  In the same place each
+// block asks for its share of dO to be brought into L2 (neutral on g2s and
+// tiestress, long step ~2420 -> ~2375 us over three runs).  The one kernel of this
 // library that reads the accumulator, the dQ convert of an earlier call, lets
 // its dependents start only after its last read.
 // 8 consecutive elements of O as they sit in memory (16 bytes of bf16 or
@@ -119,6 +121,17 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
     for (long long i = lo + threadIdx.x; i < hi; i += blockDim.x) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     // the 256-byte block after the accumulator (the d = 128 kernel's work-item counter)
     if (blockIdx.x == 0 && threadIdx.x < 64) reinterpret_cast<unsigned int*>(dq_acc + rows * D)[threadIdx.x] = 0u;
+  }
+  // and its share of dO into L2 (a prefetch is only a hint, so it is harmless
+  // even if the previous grid is still writing dO)
+  if (threadIdx.x == 0) {
+    const long long nb = rows * D * 2;  // bytes of dO; its base is 16-byte aligned (checked by its tensor map)
+    const long long lo = (nb * blockIdx.x / gridDim.x) & ~15ll;
+    const long long hi = (blockIdx.x + 1 == gridDim.x) ? nb : ((nb * (blockIdx.x + 1) / gridDim.x) & ~15ll);
+    for (long long a = lo; a < hi; a += (1ll << 20)) {
+      const long long n = (hi - a < (1ll << 20)) ? (hi - a) : (1ll << 20);
+      bulk_prefetch_l2(reinterpret_cast<const char*>(dO) + a, static_cast<uint32_t>(n));
+    }
   }
   grid_dependency_wait();  // O comes from the forward grid
   for (long long r0 = warp_global * (RPW * U); r0 < rows; r0 += n_warps * (RPW * U)) {
