@@ -99,3 +99,38 @@ def test_workspace_shared_with_the_high_precision_backward():
     torch.cuda.synchronize(dev)
     assert fa.fa_device_error()[0] == 0
     _check_call(w, ws)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_calls_back_to_back_on_one_workspace(d):
+    """Two fa_bwd calls in a row on one stream and one workspace, with no
+    forward between them: the second call's delta kernel follows the first
+    call's dQ convert directly, and it clears the accumulator the convert
+    reads.  Both calls must match the oracle (the second has another dO, so a
+    clear that overtook the convert would show in the first call's dQ)."""
+    w1 = _workload(1, 2, 384, d, True, 21 + d)
+    rng = np.random.default_rng(99 + d)
+    do2 = workloads.to_bf16_values(rng.standard_normal(w1.do.shape).astype(np.float32))
+    w2 = workloads.Workload(f"ws{d}b", *w1.q.shape, w1.causal, 0, w1.q, w1.k, w1.v, do2, w1.forced_tie_rows)
+    dev = torch.device("cuda:0")
+    B, H, N, _ = w1.q.shape
+    q, k, v, do1 = (P.to_dev(x, dev) for x in (w1.q, w1.k, w1.v, w1.do))
+    do2_t = P.to_dev(do2, dev)
+    o, lse, st = fa.attention_forward(q, k, v, True, 1, 2.0)
+    ws = torch.full((fa.fa_bwd_workspace_bytes(B, H, N, d),), 0x5A, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+    res = []
+    for do_t in (do1, do2_t):
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        fa.fa_bwd(q, k, v, o, do_t, lse, st.m, dq, dk, dv, ws, True, 1, 2.0)
+        res.append((dq, dk, dv))
+    torch.cuda.synchronize(dev)
+    status, word = fa.fa_device_error()
+    assert status == 0, f"device error word {word:#x}"
+    o_np = o.float().cpu().numpy()
+    for w, (dq, dk, dv) in zip((w1, w2), res):
+        gpu = {"o": o_np, "lse": lse.float().cpu().numpy(), "rm": st.rm.float().cpu().numpy(),
+               "rs": st.rs.cpu().numpy(), "m": st.m.float().cpu().numpy(),
+               "dq": dq.float().cpu().numpy(), "dk": dk.float().cpu().numpy(), "dv": dv.float().cpu().numpy()}
+        ref = P.oracle(w, 1, o_gpu=o_np)
+        P.compare(gpu, ref, exact_stats=False)
