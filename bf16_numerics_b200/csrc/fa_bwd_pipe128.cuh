@@ -304,24 +304,38 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
       constexpr uint32_t IDESC_SQ = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, false, true);   // dV, dK
       constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, 128, true, true);    // dQ
-      auto q_tile = [&](int g) { return base + L::Q_OFF + (g % NST) * TILE; };
-      auto do_tile = [&](int g) { return base + L::DO_OFF + (g % NST) * TILE; };
+      // Shared-memory descriptors, built once: the start-address field holds
+      // address >> 4 in its low 14 bits and every operand lies below 256 KB,
+      // so a descriptor for (tile + offset) is the tile's descriptor plus
+      // offset >> 4 (no carry leaves the field).
+      const uint64_t dk_k = sdesc_sw128(base + L::K_OFF, 16, 1024);       // K, K-major (S^T A)
+      const uint64_t dv_k = sdesc_sw128(base + L::V_OFF, 16, 1024);       // V, K-major (dP^T A)
+      const uint64_t dq_k = sdesc_sw128(base + L::Q_OFF, 16, 1024);       // Q stage 0, K-major (S^T B)
+      const uint64_t ddo_k = sdesc_sw128(base + L::DO_OFF, 16, 1024);     // dO stage 0, K-major (dP^T B)
+      const uint64_t ddo_mn = sdesc_sw128(base + L::DO_OFF, HALF, 1024);  // dO stage 0, MN-major (dV B)
+      const uint64_t dq_mn = sdesc_sw128(base + L::Q_OFF, HALF, 1024);    // Q stage 0, MN-major (dK B)
+      const uint64_t dds_mn = sdesc_sw128(base + L::DS_OFF, HALF, 1024);  // dS, MN-major (dQ A)
+      const uint64_t dk_mn = sdesc_sw128(base + L::K_OFF, HALF, 1024);    // K, MN-major (dQ B)
+      constexpr uint64_t kStage = TILE >> 4;                              // one ring stage
+      auto ring_stage = [&](int g) -> uint64_t {
+        return kStage * static_cast<uint64_t>(static_cast<uint32_t>(g) % NST);
+      };
       // S^T = K Q_g^T and dP^T = V dO_g^T   (K-dim = d: two 64-column halves)
       auto issue_s = [&](int g) {
+        const uint64_t qb = dq_k + ring_stage(g);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
-          mma_ss(tmem + L::S_COL, sdesc_sw128(base + L::K_OFF + koff, 16, 1024),
-                 sdesc_sw128(q_tile(g) + koff, 16, 1024), IDESC_SQ, ks > 0 ? 1u : 0u);
+          const uint32_t koff = ((ks >> 2) * HALF + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + L::S_COL, dk_k + koff, qb + koff, IDESC_SQ, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(L::S_FULL));
       };
       auto issue_dp = [&](int g) {
+        const uint64_t ob = ddo_k + ring_stage(g);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
-          mma_ss(tmem + L::DP_COL, sdesc_sw128(base + L::V_OFF + koff, 16, 1024),
-                 sdesc_sw128(do_tile(g) + koff, 16, 1024), IDESC_SQ, ks > 0 ? 1u : 0u);
+          const uint32_t koff = ((ks >> 2) * HALF + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + L::DP_COL, dv_k + koff, ob + koff, IDESC_SQ, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(L::DP_FULL));
       };
@@ -349,7 +363,7 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
           // dV += P^T dO_g   (K-dim = queries; P^T at S^T cols [0,64))
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ts(tmem + L::DV_COL, tmem + L::S_COL + 8u * ks, sdesc_sw128(do_tile(g) + ks * 2048, HALF, 1024),
+            mma_ts(tmem + L::DV_COL, tmem + L::S_COL + 8u * ks, ddo_mn + ring_stage(g) + 128u * ks,
                    IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
           // S^T of the next block overwrites P^T_g after dV_g has read it
           if (i + 1 < n) {
@@ -363,14 +377,13 @@ fa_bwd_main_pipe128_kernel(const __grid_constant__ CUtensorMap tm_q, const __gri
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             const uint32_t a = tmem + L::DP_COL + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4));
-            mma_ts(tmem + L::DK_COL, a, sdesc_sw128(q_tile(g) + ks * 2048, HALF, 1024), IDESC_KV,
+            mma_ts(tmem + L::DK_COL, a, dq_mn + ring_stage(g) + 128u * ks, IDESC_KV,
                    (i > 0 || ks > 0) ? 1u : 0u);
           }
           // dQ_g = dS K into the dP^T columns (after dK_g has read dS^T there)
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + L::DP_COL, sdesc_sw128(base + L::DS_OFF + ks * 2048, HALF, 1024),
-                   sdesc_sw128(base + L::K_OFF + ks * 2048, HALF, 1024), IDESC_DQ, ks > 0 ? 1u : 0u);
+            mma_ss(tmem + L::DP_COL, dds_mn + 128u * ks, dk_mn + 128u * ks, IDESC_DQ, ks > 0 ? 1u : 0u);
           tc_commit(bar(L::DQ_FULL));
           tc_commit(bar(L::Q_EMPTY + (g % NST)));
           if (i + 1 == n) {

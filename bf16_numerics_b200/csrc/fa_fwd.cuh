@@ -324,27 +324,33 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
       // S_t = Q(buffer b, slot t) K(stage s)^T into slot t's S columns
+      // descriptor arithmetic: (tile + offset) is the tile's descriptor plus
+      // offset >> 4 (the start-address field holds address >> 4 in 14 bits
+      // and every operand lies below 256 KB, so no carry leaves the field)
+      const uint64_t dk0 = sdesc_sw128(base + L::K_OFF, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(base + L::V_OFF, L::HALF, 1024);
+      constexpr uint64_t kTile = L::TILE >> 4;
       auto issue_s = [&](int b, int t, int s) {
+        const uint64_t qa = sdesc_sw128(q_tile(b, t), 16, 1024), kb = dk0 + kTile * static_cast<uint64_t>(s);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t koff = (ks >> 2) * L::HALF + (ks & 3) * 32;
-          mma_ss(tmem + L::s_col(t), sdesc_sw128(q_tile(b, t) + koff, 16, 1024),
-                 sdesc_sw128(base + L::K_OFF + s * L::TILE + koff, 16, 1024), IDESC_S, ks > 0 ? 1u : 0u);
+          const uint32_t koff = ((ks >> 2) * L::HALF + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + L::s_col(t), qa + koff, kb + koff, IDESC_S, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(L::S_FULL + t));
       };
       // O_t (+)= P_bar_t V(stage s)  (and O_lo_t (+)= P_lo_t V)
       auto issue_pv = [&](int t, int s, bool acc) {
-        const uint32_t vbase = base + L::V_OFF + s * L::TILE;
+        const uint64_t vd = dv0 + kTile * static_cast<uint64_t>(s);
 #pragma unroll
         for (int ks = 0; ks < L::BN / 16; ++ks) {
-          const uint64_t bdesc = sdesc_sw128(vbase + ks * 2048, L::HALF, 1024);
+          const uint64_t bdesc = vd + 128u * ks;
           mma_ts(tmem + L::o_col(t), tmem + L::s_col(t) + 8u * ks, bdesc, IDESC_O, (acc || ks > 0) ? 1u : 0u);
         }
         if constexpr (HP) {
 #pragma unroll
           for (int ks = 0; ks < L::BN / 16; ++ks) {
-            const uint64_t bdesc = sdesc_sw128(vbase + ks * 2048, L::HALF, 1024);
+            const uint64_t bdesc = vd + 128u * ks;
             mma_ts(tmem + L::olo_col(t), tmem + L::s_col(t) + 64u + 8u * ks, bdesc, IDESC_O,
                    (acc || ks > 0) ? 1u : 0u);
           }

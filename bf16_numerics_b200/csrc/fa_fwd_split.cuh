@@ -289,14 +289,22 @@ fa_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
+      // Shared-memory descriptors, built once: the start-address field holds
+      // address >> 4 in its low 14 bits and every operand lies below 256 KB,
+      // so a descriptor for (tile + offset) is the tile's descriptor plus
+      // offset >> 4 (no carry leaves the field).
+      const uint64_t dq0 = sdesc_sw128(base + L::Q_OFF, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(base + L::K_OFF, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(base + L::V_OFF, L::HALF, 1024);
+      constexpr uint64_t kTile = L::TILE >> 4;
       // S(g) = Q(buffer qs) K(stage g&1)^T into the single S slot
       auto issue_s = [&](int qs, int g) {
         const int s = g & 1;
+        const uint64_t qa = dq0 + kTile * static_cast<uint64_t>(qs), kb = dk0 + kTile * static_cast<uint64_t>(s);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t koff = (ks >> 2) * L::HALF + (ks & 3) * 32;
-          mma_ss(tmem + L::S_COL, sdesc_sw128(base + L::Q_OFF + qs * L::TILE + koff, 16, 1024),
-                 sdesc_sw128(base + L::K_OFF + s * L::TILE + koff, 16, 1024), IDESC_S, ks > 0 ? 1u : 0u);
+          const uint32_t koff = ((ks >> 2) * L::HALF + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + L::S_COL, qa + koff, kb + koff, IDESC_S, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(L::S_FULL));
         tc_commit(bar(L::K_EMPTY + s));
@@ -328,16 +336,16 @@ fa_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           if (!wait(bar(L::P_FULL), gt & 1, 7)) { ok = false; break; }
           if (!wait(bar(L::V_FULL + (gt & 1)), (gt >> 1) & 1, 8)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t vbase = base + L::V_OFF + (gt & 1) * L::TILE;
+          const uint64_t vd = dv0 + kTile * static_cast<uint64_t>(gt & 1);
 #pragma unroll
           for (int ks = 0; ks < L::BN / 16; ++ks) {
-            const uint64_t b = sdesc_sw128(vbase + ks * 2048, L::HALF, 1024);
+            const uint64_t b = vd + 128u * ks;
             mma_ts(tmem + L::O_COL, tmem + L::P_COL + 8u * ks, b, IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
           }
           if constexpr (HP) {
 #pragma unroll
             for (int ks = 0; ks < L::BN / 16; ++ks) {
-              const uint64_t b = sdesc_sw128(vbase + ks * 2048, L::HALF, 1024);
+              const uint64_t b = vd + 128u * ks;
               mma_ts(tmem + L::OLO_COL, tmem + L::PLO_COL + 8u * ks, b, IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
             }
           }
