@@ -21,7 +21,9 @@
 //     warpgroup has just read (64h + [0,32)).
 //   * dQ_g = dS K is one N = 64 product into S^T cols [64,128) of the same
 //     buffer, issued after dV_g has read P^T there (products from one thread
-//     run in issue order); no later product of the block touches it.
+//     run in issue order); no later product of the block touches it.  It
+//     goes ahead of dK_g, so the drain can release the buffer for S^T of
+//     block g+2 sooner (g2s step 119.4 -> 118.4 us).
 //   * Four drain warps move the dQ partial from TMEM into a 128B-swizzled
 //     fp32 staging box in shared memory and add it to the fp32 accumulator in
 //     global memory with one TMA tensor reduce-add per 32-column half, one
@@ -45,6 +47,8 @@
 // instructions count: its shared-memory descriptors are built once and
 // advanced by constants, and its warpgroup gets the registers that keep it
 // from spilling (measured on g2s: backward 68.1 -> 66.3 us for the two).
+// Each descriptor is passed as two 32-bit halves, the high half a constant of
+// the layout, so advancing one costs a single 32-bit add.
 #pragma once
 
 #include "fa_bwd.cuh"
@@ -256,30 +260,28 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       constexpr uint32_t IDESC_SQ = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 64, false, true);    // dV, dK
       constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, 64, true, true);     // dQ
-      // Shared-memory descriptors, built once: the start-address field holds
-      // address >> 4 in its low 14 bits and every operand lies below 256 KB,
-      // so a descriptor for (tile + offset) is the tile's descriptor plus
-      // offset >> 4 (no carry leaves the field).
-      const uint64_t dk_k = sdesc_sw128(base + L::K_OFF, 16, 1024);        // K, K-major (S^T A)
-      const uint64_t dv_k = sdesc_sw128(base + L::V_OFF, 16, 1024);        // V, K-major (dP^T A)
-      const uint64_t dq_k = sdesc_sw128(base + L::Q_OFF, 16, 1024);        // Q stage 0, K-major (S^T B)
-      const uint64_t ddo_k = sdesc_sw128(base + L::DO_OFF, 16, 1024);      // dO stage 0, K-major (dP^T B)
-      const uint64_t ddo_mn = sdesc_sw128(base + L::DO_OFF, 16384, 1024);  // dO stage 0, MN-major (dV B)
-      const uint64_t dq_mn = sdesc_sw128(base + L::Q_OFF, 16384, 1024);    // Q stage 0, MN-major (dK B)
-      const uint64_t dds_mn = sdesc_sw128(base + L::DS_OFF, 16384, 1024);  // dS, MN-major (dQ A)
-      const uint64_t dk_mn = sdesc_sw128(base + L::K_OFF, 16384, 1024);    // K, MN-major (dQ B)
-      constexpr uint64_t kStage = TILE >> 4;                               // one ring stage
+      // Shared-memory descriptors, built once, as two 32-bit halves.  The low
+      // half holds address >> 4 in 14 bits and the leading byte offset; every
+      // operand lies below 256 KB, so the descriptor of (tile + offset) is the
+      // tile's low half plus offset >> 4 (no carry leaves the field).  The
+      // high half is a constant of the layout (stride 1024, version, swizzle).
+      constexpr uint32_t HI = (1024u >> 4) | (1u << 14) | (2u << 29);
+      const uint32_t lo_k = static_cast<uint32_t>(sdesc_sw128(base, 16, 1024));      // K-major, offset 0
+      const uint32_t lo_mn = static_cast<uint32_t>(sdesc_sw128(base, 16384, 1024));  // MN-major, offset 0
+      constexpr uint32_t kStage = TILE >> 4;                                        // one ring stage
       auto issue_s = [&](int g) {
         const uint32_t d_tmem = tmem + 128u * (g & 1);
-        const uint64_t qb = dq_k + kStage * static_cast<uint64_t>(g % NST);
+        const uint32_t qb = lo_k + (L::Q_OFF >> 4) + kStage * static_cast<uint32_t>(g % NST);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) mma_ss(d_tmem, dk_k + 2u * ks, qb + 2u * ks, IDESC_SQ, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ss2(d_tmem, lo_k + (L::K_OFF >> 4) + 2u * ks, HI, qb + 2u * ks, HI, IDESC_SQ, ks > 0 ? 1u : 0u);
         tc_commit(bar(L::S_FULL + (g & 1)));
       };
       auto issue_dp = [&](int g) {
-        const uint64_t ob = ddo_k + kStage * static_cast<uint64_t>(g % NST);
+        const uint32_t ob = lo_k + (L::DO_OFF >> 4) + kStage * static_cast<uint32_t>(g % NST);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) mma_ss(tmem + L::DPT_COL, dv_k + 2u * ks, ob + 2u * ks, IDESC_SQ, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ss2(tmem + L::DPT_COL, lo_k + (L::V_OFF >> 4) + 2u * ks, HI, ob + 2u * ks, HI, IDESC_SQ, ks > 0 ? 1u : 0u);
         tc_commit(bar(L::DP_FULL));
       };
       BwdCursor cur;
@@ -311,24 +313,25 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           // dV += P^T dO_g   (K-dim = queries; P^T at S^T cols [0,32) and [64,96))
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ts(tmem + L::DV_COL, tmem + 128u * b + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4)),
-                   ddo_mn + kStage * static_cast<uint64_t>(g % NST) + 128u * ks,
-                   IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
+            mma_ts2(tmem + L::DV_COL, tmem + 128u * b + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4)),
+                    lo_mn + (L::DO_OFF >> 4) + kStage * static_cast<uint32_t>(g % NST) + 128u * ks, HI,
+                    IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
           if (!wait(bar(L::DS_FULL), g & 1, 5)) { ok = false; break; }
           FA_TRACE_POINT(11);
           tc_fence_after();
+          // dQ_g = dS K into S^T cols [64,128) of the same buffer
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ss2(tmem + 128u * b + 64u, lo_mn + (L::DS_OFF >> 4) + 128u * ks, HI, lo_mn + (L::K_OFF >> 4) + 128u * ks,
+                    HI, IDESC_DQ, ks > 0 ? 1u : 0u);
+          tc_commit(bar(L::DQ_FULL + b));  // the drain may take dQ_g while dK_g runs
           // dK += dS^T Q_g
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             const uint32_t a = tmem + L::DPT_COL + (ks < 4 ? 8u * ks : 64u + 8u * (ks - 4));
-            mma_ts(tmem + L::DK_COL, a, dq_mn + kStage * static_cast<uint64_t>(g % NST) + 128u * ks, IDESC_KV,
-                   (i > 0 || ks > 0) ? 1u : 0u);
+            mma_ts2(tmem + L::DK_COL, a, lo_mn + (L::Q_OFF >> 4) + kStage * static_cast<uint32_t>(g % NST) + 128u * ks,
+                    HI, IDESC_KV, (i > 0 || ks > 0) ? 1u : 0u);
           }
-          // dQ_g = dS K into S^T cols [64,128) of the same buffer
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + 128u * b + 64u, dds_mn + 128u * ks, dk_mn + 128u * ks, IDESC_DQ, ks > 0 ? 1u : 0u);
-          tc_commit(bar(L::DQ_FULL + b));
           tc_commit(bar(L::Q_EMPTY + (g % NST)));
           if (i + 1 < n) {
             issue_dp(g + 1);
