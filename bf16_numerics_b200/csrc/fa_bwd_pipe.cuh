@@ -87,6 +87,11 @@ struct BwdPipeLayout {
   static constexpr int THREADS = 512;
   static constexpr uint32_t REGS_ELEM = 160, REGS_DRAIN = 88, REGS_CTRL = 104;
 };
+// setmaxnreg draws on the registers the block was launched with (512 threads
+// x 128): a split above that total would wait forever
+static_assert(2 * BwdPipeLayout::REGS_ELEM + BwdPipeLayout::REGS_DRAIN + BwdPipeLayout::REGS_CTRL == 4 * 128,
+              "register split");
+static_assert(BwdPipeLayout::SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int x, int y, int z) {
   asm volatile(

@@ -93,6 +93,10 @@ struct BwdPipe128Layout {
   static constexpr uint32_t REGS_ELEM = 168, REGS_DRAIN = 88, REGS_CTRL = 88;
 };
 static_assert(BwdPipe128Layout::SMEM_BYTES <= 227 * 1024, "shared memory budget");
+// setmaxnreg draws on the registers the block was launched with (512 threads
+// x 128): a split above that total would wait forever
+static_assert(2 * BwdPipe128Layout::REGS_ELEM + BwdPipe128Layout::REGS_DRAIN + BwdPipe128Layout::REGS_CTRL == 4 * 128,
+              "register split");
 
 // Work item number w -> (key block, batch*head).  Items come in groups of
 // head_group heads (the last group may be smaller); inside a group, key block

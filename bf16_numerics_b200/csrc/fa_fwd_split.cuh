@@ -74,6 +74,12 @@ struct FwdSplitLayout {
   static constexpr uint32_t REGS_SOFT = 104, REGS_CTRL = 32;
 };
 
+// setmaxnreg draws on the registers the block was launched with (two CTAs
+// per SM: 384 threads x 80): a split above that total would wait forever
+static_assert(2 * FwdSplitLayout<64, false>::REGS_SOFT + FwdSplitLayout<64, false>::REGS_CTRL == 3 * 80,
+              "register split");
+static_assert(2 * FwdSplitLayout<64, false>::SMEM_BYTES <= 228 * 1024, "two CTAs per SM");
+
 // The work items of one CTA, in order (see the file comment).  Only the
 // item's coordinates are held; the rest is read from the launch (kernel
 // parameters and the grid shape) when needed.
