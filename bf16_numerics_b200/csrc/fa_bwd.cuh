@@ -25,8 +25,8 @@
 //   S^T  = K  Q_i^T   (A: K  smem K-major, B: Q_i  smem K-major)
 //   dP^T = V  dO_i^T  (A: V  smem K-major, B: dO_i smem K-major)
 //   dV  += P^T  dO_i  (A: P^T  TMEM,     B: dO_i smem MN-major, N = d)
-//   dK  += dS^T Q_i   (A: dS^T from TMEM (d = 128) or from the shared-memory
-//                      dS tile read K-major (d = 64), B: Q_i smem MN-major, N = d)
+//   dK  += dS^T Q_i   (A: dS^T from TMEM, written over dP^T columns the
+//                      elementwise warps have read, B: Q_i smem MN-major, N = d)
 //   dQ_i = dS   K     (A: dS smem MN-major (written from dS^T), B: K MN-major)
 #pragma once
 
