@@ -191,7 +191,11 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     tmem_relinquish();
   }
   grid_launch_dependents();
-  grid_dependency_wait();  // delta and the cleared dQ accumulator come from the previous grid
+  // No dependency wait here: the delta kernel before this one lets it launch
+  // only once every earlier grid in the stream has completed, so Q, K, V, dO,
+  // lse and the shift are final.  Only delta and the cleared dQ accumulator
+  // come from the delta grid itself; the drain warps, which read the one and
+  // add into the other, wait for it.
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -399,6 +403,7 @@ fa_bwd_main_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       sts32(base + L::VEC_OFF + ((s * 2 + 1) * 128 + t) * 4, dl);
       mbar_arrive(bar(L::VEC_FULL + s));
     };
+    grid_dependency_wait();  // delta and the cleared dQ accumulator: the delta grid's
     // pub walks two blocks ahead of cur, nxt holds the loads for pub
     BwdCursor cur, pub;
     cur.start(p);
