@@ -46,11 +46,16 @@ namespace fa {
 // (two per SM, 80 registers x 384 threads each), so with programmatic
 // dependent launch they are resident when the forward ends (measured: g2s
 // step 123.0 -> 122.4 us, long 2415 -> 2392 us, against 256-thread blocks).
-// The clear does not depend on the forward: every block zeroes its own
-// contiguous share of the accumulator before it waits for the forward grid,
-// so the blocks resident beside the forward's CTAs clear theirs while it
-// runs (measured against clearing each block's rows in the dot loop: g2s
-// step 123.1 -> 121.3 us, long 2396 -> 2373 us).  In the same place each
+// The clear does not depend on the forward: the first clear_blocks blocks
+// zero one contiguous share of the accumulator each before they wait for the
+// forward grid.  When the accumulator is small (a quarter of L2 at most) the
+// host makes that one block per SM, the blocks resident beside the forward's
+// CTAs, so the whole clear runs while the forward does (g2s step 116.7 ->
+// 115.7 us); a larger one is shared by every block, since clearing it beside
+// the forward would push the forward's K and V tiles out of L2 (long: 2546
+// against 2373 us).  Against clearing each block's rows in the dot loop the
+// shared form took the g2s step from 123.1 to 121.3 us and long from 2396 to
+// 2373 us.  In the same place each
 // block asks for its share of dO to be brought into L2 (neutral on g2s and
 // tiestress, long step ~2420 -> ~2375 us over three runs).  The one kernel of this
 // library that reads the accumulator, the dQ convert of an earlier call, lets
@@ -105,7 +110,7 @@ struct ORaw<float> {
 template <int D, typename OT>
 __global__ void __launch_bounds__(128, 16)
 fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
-                    float* __restrict__ delta, float* __restrict__ dq_acc, long long rows) {
+                    float* __restrict__ delta, float* __restrict__ dq_acc, long long rows, int clear_blocks) {
   constexpr int LPR = D / 8;               // lanes per row (8 elements per lane)
   constexpr int RPW = 32 / LPR;            // rows per warp per group
   constexpr int U = 2;                     // row groups per warp per pass
@@ -113,9 +118,9 @@ fa_bwd_delta_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ 
   const long long warp_global = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const int sub = lane / LPR, li = lane % LPR;
-  {
+  if (static_cast<int>(blockIdx.x) < clear_blocks) {
     const long long n4 = rows * (D / 4);
-    const long long lo = n4 * blockIdx.x / gridDim.x, hi = n4 * (blockIdx.x + 1) / gridDim.x;
+    const long long lo = n4 * blockIdx.x / clear_blocks, hi = n4 * (blockIdx.x + 1) / clear_blocks;
     float4* acc4 = reinterpret_cast<float4*>(dq_acc);
     for (long long i = lo + threadIdx.x; i < hi; i += blockDim.x) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     // the 256-byte block after the accumulator (the d = 128 kernel's work-item counter)

@@ -189,6 +189,31 @@ int sm_count() {
   return cached[dev].load();
 }
 
+// L2 size of the current device in bytes (queried once per device; 0 if unknown).
+long long l2_bytes() {
+  static std::atomic<long long> cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrL2CacheSize, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev].load();
+}
+
+// How many delta blocks clear the dQ accumulator (before their dependency
+// wait).  A small accumulator, a quarter of L2 at most, goes to one block per
+// SM: those blocks sit beside the forward's CTAs and clear it while the
+// forward runs.  A larger one is shared by every block, because clearing it
+// beside the forward would push the forward's K and V tiles out of L2.
+int delta_clear_blocks(int grid, long long acc_bytes) {
+  const int n_sm = sm_count();
+  const long long l2 = l2_bytes();
+  if (n_sm <= 0 || l2 <= 0 || acc_bytes > l2 / 4 || grid <= n_sm) return grid;
+  return n_sm;
+}
+
 bool shape_ok(int B, int H, int N, int d) {
   if (B < 0 || H < 0 || N < 0) return false;
   const long long BH = static_cast<long long>(B) * H;
@@ -304,12 +329,14 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     constexpr int rows_per_block = 4 * (32 / (D / 8)) * 2;  // 4 warps x rows per group x 2 groups
     LaunchTimer tm(FA_KERNEL_BWD_DELTA, stream);
     const dim3 grid(grid_for(rows, rows_per_block));
+    const int clear_blocks = delta_clear_blocks(static_cast<int>(grid.x), static_cast<long long>(acc_bytes));
     cudaError_t e =
         o_is_hp ? launch_pdl(fa::fa_bwd_delta_kernel<D, float>, grid, dim3(128), 0, stream,
-                             static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows)
+                             static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows,
+                             clear_blocks)
                 : launch_pdl(fa::fa_bwd_delta_kernel<D, __nv_bfloat16>, grid, dim3(128), 0, stream,
                              static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta,
-                             dq_acc, rows);
+                             dq_acc, rows, clear_blocks);
     tm.done();
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("fa_bwd_delta_kernel launch", e);
