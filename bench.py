@@ -154,10 +154,11 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- oracle arm
-def cpu_oracle_sample(w, mode, beta, seconds):
+def cpu_oracle_sample(w, mode, beta, seconds, first=None):
     """Time the float64 oracle fwd+bwd on (batch, head) pairs, in order and
     wrapping around to the first head, until about `seconds` of CPU work;
-    returns (flops_done, elapsed, head evaluations, threads)."""
+    returns (flops_done, elapsed, head evaluations, threads).  If `first` is a
+    dict, the first head's results (o, dq, dk, dv) are stored in it."""
     from oracle import attention as A
     from threadpoolctl import threadpool_info
 
@@ -167,13 +168,29 @@ def cpu_oracle_sample(w, mode, beta, seconds):
     while True:
         sub = w.heads([pairs[done % len(pairs)]])
         f = A.attention_fwd(sub.q, sub.k, sub.v, sub.causal, mode, beta)
-        A.attention_bwd(sub.q, sub.k, sub.v, sub.do, sub.causal, mode, beta, fwd=f)
+        g = A.attention_bwd(sub.q, sub.k, sub.v, sub.do, sub.causal, mode, beta, fwd=f)
+        if first is not None and done == 0:
+            first.update(o=f["o"], dq=g["dq"], dk=g["dk"], dv=g["dv"])
         done += 1
         if time.perf_counter() - t0 >= seconds:
             break
     elapsed = time.perf_counter() - t0
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     return per_head * done, elapsed, done, threads
+
+
+def parity_readout(ref, gpu):
+    """Max-abs error / max|ref| of head (0, 0) for each output: GPU against
+    the float64 oracle chained forward -> backward."""
+    import numpy as np
+
+    out = {"head": "(b, h) = (0, 0)", "reference": "float64 oracle, its own O in the backward",
+           "bar": 1e-2}
+    for key in ("o", "dq", "dk", "dv"):
+        r = np.asarray(ref[key], dtype=np.float64).reshape(-1)
+        g_ = gpu[key][0, 0].float().cpu().numpy().astype(np.float64).reshape(-1)
+        out[key] = float(np.abs(g_ - r).max() / max(np.abs(r).max(), 1e-30))
+    return out
 
 
 # ------------------------------------------------------------------ ranks
@@ -251,7 +268,7 @@ def workload_config(w, mode, beta):
             "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
             "softmax_mode": MODE_TEXT[mode], "beta": beta,
             "l2": "flushed before every timed step (256 MiB write, then a 256 MiB read of another buffer; outside the timed intervals)",
-            "inputs": inputs}
+            "inputs": inputs, "seed": w.seed}
 
 
 def run_reference(args, rank, world):
@@ -489,11 +506,15 @@ def run_ours(args, rank, world, local_rank):
                     "serial_value": e2e_serial},
             "clocks": clocks, "step_ms_p10_p50_p90": [float(np.percentile(step_ms, p)) for p in (10, 50, 90)]}
     if world == 1 and not args.no_cpu_baseline:
-        flops_c, secs_c, heads_c, threads_c = cpu_oracle_sample(w, mode, beta, args.cpu_seconds)
+        first = {}
+        flops_c, secs_c, heads_c, threads_c = cpu_oracle_sample(w, mode, beta, args.cpu_seconds, first)
         line["cpu_baseline"] = {"value": flops_c / secs_c / 1e12, "unit": "TFLOP/s", "cores": threads_c,
                                 "kind": "oracle",
                                 "sample": f"{heads_c} (b,h)-head fwd+bwd evaluations cycling over the {B * H} heads "
                                           f"of the same workload, float64 NumPy oracle, {secs_c:.1f} s"}
+        # the oracle's first head against the GPU's outputs for it (the last
+        # timed step's inputs are the workload's, so the outputs are too)
+        line["parity"] = parity_readout(first, {"o": o, "dq": dq, "dk": dk, "dv": dv})
     print(json.dumps(line), flush=True)
     return 0
 

@@ -1,7 +1,10 @@
 """Host-side logic of bench.py on the CPU: the per-workload DRAM traffic
-record, the clock/throttle-reason parsing and the peaks fallback."""
+record, the clock/throttle-reason parsing, the peaks fallback and the parity
+readout."""
 
 import os
+
+import numpy as np
 
 import bench
 
@@ -99,3 +102,20 @@ def test_every_launched_kernel_has_its_roofline():
                  ("fa_fwd_kernel", "fa_bwd_delta_kernel", "fa_bwd_main_kernel", "fa_bwd_dq_convert_kernel")]
         assert [bench.kernel_bound(n) for n in names] == ["tensor", "hbm", "tensor", "hbm"]
         assert [bench.kernel_role(n) for n in names] == ["fwd", "delta", "bwd_main", "dq_convert"]
+
+
+def test_parity_readout_is_relative_max_abs_error_of_head_zero():
+    """bench.py's parity field: max-abs error / max|ref| of head (0, 0) for O,
+    dQ, dK, dV, the GPU side read through float32."""
+    import torch
+
+    rng = np.random.default_rng(3)
+    ref = {key: rng.standard_normal((1, 1, 16, 8)) for key in ("o", "dq", "dk", "dv")}
+    gpu = {key: torch.from_numpy(ref[key]).float() for key in ref}
+    same = bench.parity_readout(ref, gpu)
+    assert all(same[key] < 1e-6 for key in ("o", "dq", "dk", "dv"))
+    assert same["bar"] == 1e-2
+    bump = dict(gpu)
+    bump["dk"] = gpu["dk"].clone()
+    bump["dk"][0, 0, 3, 2] += 0.25 * float(np.abs(ref["dk"]).max())
+    assert abs(bench.parity_readout(ref, bump)["dk"] - 0.25) < 1e-6
