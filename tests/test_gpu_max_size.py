@@ -1,0 +1,106 @@
+"""Problems past 2^31 elements per tensor (GPU).
+
+B*H*N*d is just above 2^31, so in the last heads every element offset into
+Q, K, V, O, dO, dQ, dK, dV and the fp32 dQ accumulator passes 2^31 (and every
+byte offset of the accumulator passes 2^33).  The library accepts any
+B*H*N*d below 2^40; this checks that its kernels' offsets, the delta/clear
+and convert kernels' grid-stride loops and the tensor maps hold there.
+
+The heads compared with the oracle sit at the start, on both sides of 2^30
+elements (2^31 bytes of a bf16 tensor, 2^32 of the accumulator), on both
+sides of 2^31 elements, and at the very end of the buffers.  Their inputs come
+from the named workload's construction (seeded, on the host); every other head
+holds seeded normal values drawn on the device by torch's generator, which
+only fill the problem to its size: a head's outputs depend on its own inputs
+alone.  Over the whole problem, properties that hold at any size are checked
+on the device: finite outputs, a tie count of at least one on every row, and
+the stabilised shift's bound P_bar < 1 on every tied row.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import bf16_numerics_b200 as fa
+import workloads
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+N = 1024
+H = 16
+MODE = fa.STABILIZED
+
+
+def _shape(d):
+    per_head = N * d
+    BH = (1 << 31) // per_head + H  # at least one batch entry past 2^31 elements
+    B = -(-BH // H)
+    return B, B * H, per_head
+
+
+def _bytes_needed(B, d):
+    E = B * H * N * d
+    rows = B * H * N
+    return 8 * 2 * E + fa.fa_bwd_workspace_bytes(B, H, N, d) + 5 * 4 * rows
+
+
+@pytest.mark.parametrize("d,name", [(64, "g2s"), (128, "long")])
+def test_problem_past_2_31_elements(cuda_device, d, name):
+    dev = cuda_device
+    B, BH, per_head = _shape(d)
+    assert BH * per_head > (1 << 31)
+    free, _ = torch.cuda.mem_get_info(dev)
+    need = _bytes_needed(B, d)
+    if free < need + (4 << 30):
+        pytest.skip(f"needs {need / 2**30:.1f} GiB free, {free / 2**30:.1f} GiB available")
+
+    at = lambda elem: elem // per_head  # the head holding element `elem`
+    sample = sorted({0, at(1 << 30) - 1, at(1 << 30), at(1 << 31) - 1, at(1 << 31), BH - 1})
+    small = workloads.make(name, seed=11 + d, B=1, H=len(sample), N=N)
+
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + d)
+
+    def big(x_small):
+        t = torch.randn((B, H, N, d), generator=gen, device=dev, dtype=torch.bfloat16)
+        flat = t.view(BH, N, d)
+        for j, bh in enumerate(sample):
+            flat[bh].copy_(P.to_dev(x_small[0, j], dev))
+        return t
+
+    q, k, v, do = big(small.q), big(small.k), big(small.v), big(small.do)
+    o, lse, st = fa.attention_forward(q, k, v, small.causal, MODE, 2.0)
+    dq, dk, dv, ws = fa.attention_backward(q, k, v, o, do, lse, st.m, small.causal, MODE, 2.0)
+    torch.cuda.synchronize(dev)
+    status, word = fa.fa_device_error()
+    assert status == 0, f"device error word {word:#x}"
+
+    # properties of every row and element
+    for key, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv), ("lse", lse)):
+        assert bool(torch.isfinite(t).all()), key
+    assert bool((st.rs >= 1).all())
+    tied = st.rs > 1
+    assert bool((st.pbar_max[tied] < 1.0).all())
+    assert bool((st.pbar_max[~tied] == 1.0).all())
+
+    # the sampled heads against the oracle
+    off_delta, _ = fa.fa_bwd_workspace_offsets(B, H, N, d)
+    delta = ws[off_delta:off_delta + BH * N * 4].view(torch.float32).view(BH, N)
+    idx = torch.tensor(sample, device=dev)
+
+    def pick(t, per_row):
+        flat = t.reshape(BH, N) if per_row else t.reshape(BH, N, d)
+        x = flat.index_select(0, idx)[None]
+        return x.cpu().numpy() if x.dtype == torch.int32 else x.float().cpu().numpy()
+
+    gpu = {key: pick(t, False) for key, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv))}
+    gpu.update({key: pick(t, True) for key, t in (("lse", lse), ("rm", st.rm), ("rs", st.rs), ("m", st.m),
+                                                   ("delta", delta))})
+    del q, k, v, do, o, lse, st, dq, dk, dv, ws, delta, tied
+    torch.cuda.empty_cache()
+
+    ref = P.oracle(small, MODE, o_gpu=gpu["o"])
+    errs = P.compare(gpu, ref, exact_stats=False)
+    print(f"d={d} B={B} H={H} heads {sample}:", {key: tuple(round(x, 5) for x in val) for key, val in errs.items()})
+    assert np.all(gpu["rs"][small.forced_tie_rows] >= 2)
