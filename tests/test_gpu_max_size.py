@@ -1,5 +1,7 @@
-"""Problems past 2^31 elements per tensor (GPU).
+"""Maximum sizes (GPU): problems past 2^31 elements per tensor, and rows of
+64K keys.
 
+Past 2^31 elements.
 B*H*N*d is just above 2^31, so in the last heads every element offset into
 Q, K, V, O, dO, dQ, dK, dV and the fp32 dQ accumulator passes 2^31 (and every
 byte offset of the accumulator passes 2^33).  The library accepts any
@@ -15,7 +17,20 @@ only fill the problem to its size: a head's outputs depend on its own inputs
 alone.  Over the whole problem, properties that hold at any size are checked
 on the device: finite outputs, a tie count of at least one on every row, and
 the stabilised shift's bound P_bar < 1 on every tied row.
+
+Rows of 64K keys.  A non-causal problem of n = 1024 rows whose Q, K, V and
+dO are repeated r = 64 times along the sequence (N = 65536) has, row for row,
+the small problem's outputs: each key appears r times, so every softmax
+weight is the small problem's divided by r, and the r copies of a key or of a
+query collect the same sums (O, dQ, dK and dV are unchanged, lse grows by
+ln r, the row maximum is unchanged and its tie count is r times the small
+one's, so every row is tied and the shift rule takes its tied branch).  The
+oracle runs on the small problem; the GPU runs the whole long one (512 key
+tiles per row, 512 query blocks adding into every dQ block).
 """
+
+import dataclasses
+import math
 
 import numpy as np
 import pytest
@@ -23,6 +38,7 @@ import torch
 
 import bf16_numerics_b200 as fa
 import workloads
+from oracle import attention as A
 from tests import parity as P
 
 pytestmark = pytest.mark.gpu
@@ -104,3 +120,31 @@ def test_problem_past_2_31_elements(cuda_device, d, name):
     errs = P.compare(gpu, ref, exact_stats=False)
     print(f"d={d} B={B} H={H} heads {sample}:", {key: tuple(round(x, 5) for x in val) for key, val in errs.items()})
     assert np.all(gpu["rs"][small.forced_tie_rows] >= 2)
+
+
+REPEAT = 64
+
+
+@pytest.mark.parametrize("d,name,mode", [(64, "tiestress", 0), (64, "tiestress", 1), (128, "long", 1)])
+def test_rows_of_64k_keys_by_repetition(cuda_device, d, name, mode):
+    small = dataclasses.replace(workloads.make(name, seed=21 + d, B=1, H=1, N=1024), causal=False)
+    n, r = small.N, REPEAT
+    rep = lambda x: np.ascontiguousarray(np.tile(x, (1, 1, r, 1)))
+    big = workloads.Workload(f"{name}x{r}", 1, 1, n * r, d, False, small.seed, rep(small.q), rep(small.k),
+                             rep(small.v), rep(small.do), np.tile(small.forced_tie_rows, (1, 1, r)))
+    gpu = P.run_gpu(big, mode, dev=cuda_device)
+    for key in ("o", "dq", "dk", "dv", "lse"):
+        assert np.all(np.isfinite(gpu[key])), key
+    assert np.all(gpu["rs"] >= r)
+    if mode == 1:
+        assert np.all(gpu["pbar_max"] < 1.0)  # every row is tied
+    for c in (0, r - 1):  # the first and the last copy of every query and key
+        rows = slice(c * n, (c + 1) * n)
+        part = {key: val[:, :, rows] for key, val in gpu.items()}
+        ref = P.oracle(small, mode, o_gpu=part["o"])
+        ref["rs"] = r * ref["rs"]
+        ref["lse"] = ref["lse"] + math.log(r)
+        ref["m"] = A.select_shift(ref["rm"], ref["rs"], 2.0, mode)
+        errs = P.compare(part, ref, exact_stats=(name == "tiestress"))
+        print(f"{name} d={d} mode {mode} N={n * r} copy {c}:",
+              {key: tuple(round(x, 5) for x in val) for key, val in errs.items()})

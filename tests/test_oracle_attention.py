@@ -185,6 +185,30 @@ def test_mode_invariance(name):
         assert np.linalg.norm(x1 - x0) <= 1e-12 * np.linalg.norm(x0)
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+def test_repeated_sequence_invariance(mode):
+    """Q, K, V, dO repeated r times along the sequence (non-causal): every
+    softmax weight is divided by r and each key's r copies share the mass, so
+    O, dQ, dK, dV are those of one copy, lse grows by ln r, rm is unchanged
+    and rs is multiplied by r (every row becomes tied)."""
+    n, r = 48, 4
+    rng = np.random.default_rng(17)
+    q, k, v, do = (_rand_bf16(rng, (1, 2, n, 16)) for _ in range(4))
+    rep = lambda x: np.tile(x, (1, 1, r, 1))
+    f = A.attention_fwd(q, k, v, False, mode, 2.0)
+    b = A.attention_bwd(q, k, v, do, False, mode, 2.0, fwd=f)
+    fr = A.attention_fwd(rep(q), rep(k), rep(v), False, mode, 2.0)
+    br = A.attention_bwd(rep(q), rep(k), rep(v), rep(do), False, mode, 2.0, fwd=fr)
+    for c in range(r):
+        rows = slice(c * n, (c + 1) * n)
+        for x, xr in ((f["o"], fr["o"]), (b["dq"], br["dq"]), (b["dk"], br["dk"]), (b["dv"], br["dv"])):
+            np.testing.assert_allclose(xr[:, :, rows], x, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(fr["lse"][:, :, rows], f["lse"] + math.log(r), rtol=0, atol=1e-12)
+        assert np.array_equal(fr["rm"][:, :, rows], f["rm"])
+        assert np.array_equal(fr["rs"][:, :, rows], r * f["rs"])
+        assert np.array_equal(fr["m"][:, :, rows], A.select_shift(f["rm"], r * f["rs"], 2.0, mode))
+
+
 # ------------------------------------------- the trigger and the fix (pages)
 
 def test_trigger_exact_ones_standard_mode():
